@@ -1,0 +1,430 @@
+"""Benchmark of one AsyncTLS decode step (two-level sparse attention) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = block score + top-K_b, label-channel token score + top-K_t, and
+sparse attention with log-sum-exp merge, for all B x H_q heads of one layer,
+through the C ABI of libtls.so.  Default workload: GQA, batch 8, 32/8 heads,
+head_dim 128, 96k context, K_b 256, K_t 4096, r 16, bf16.  Inputs are seeded
+synthetic tensors (see two_level_sparse_quest_b200/workloads.py); the step
+rotates over 4 layer copies held in separate device memory, so consecutive
+steps never hit the 126 MB L2 with the previous step's bytes.
+
+Prints one JSON line (rank 0).  Multi-GPU (torchrun): every rank runs its own
+copy of the workload (independent sequences, no collective on the data path);
+time is the max over ranks; value = steps of all ranks / time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "sparse-attn decode steps/sec (all heads) at 96k ctx; achieved HBM GB/s vs peak"
+N_LAYERS = 4
+SMI_FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+# ----------------------------------------------------------------------------- bytes
+def algorithmic_bytes(w) -> dict:
+    """Bytes one step must touch (the method's data, not scratch):
+    block summary of every block, label slab rows of the K_b * bs candidates,
+    K and V rows of the K_t kept tokens, q, out (fp32), lse, and the int32
+    block / token index lists (written once, read once)."""
+    e = w.elem_bytes
+    G = w.batch * w.n_kv_heads
+    vrow = 0 if w.v_is_k_prefix else w.d_v
+    parts = {
+        "block_summary": G * w.n_blocks * 2 * w.d_qk * e,
+        "label_slab": G * w.k_b * w.block_size * w.n_label * e,
+        "gathered_kv": G * w.k_t * (w.d_qk + vrow) * e,
+        "q": w.batch * w.n_q_heads * w.d_qk * e,
+        "out_lse": w.batch * w.n_q_heads * (w.d_v * 4 + 4),
+        "indices": G * (w.k_b + w.k_t) * 4 * 2,
+    }
+    parts["total"] = sum(parts.values())
+    # per stage (what each C call must read/write)
+    parts["stage_block"] = parts["block_summary"] + parts["q"] + G * w.k_b * 4
+    parts["stage_token"] = parts["label_slab"] + parts["q"] + G * (w.k_b + w.k_t) * 4
+    parts["stage_attn"] = parts["gathered_kv"] + parts["q"] + parts["out_lse"] + G * w.k_t * 4
+    return parts
+
+
+# ----------------------------------------------------------------------------- helpers
+def read_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "two_level_sparse_quest_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def read_traffic(stage: str):
+    """DRAM traffic per launch from a committed ncu summary, only if it was
+    taken on the kernel sources as they are now."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    ent = d.get(stage)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={SMI_FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
+                 "-i", str(self.gpu)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            threading.Thread(target=self._read, daemon=True).start()
+            time.sleep(0.5)
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self) -> dict:
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons, power = [], [], set(), []
+        for ts, line in self.lines:
+            if self.t0 and (ts < self.t0 or ts > (self.t1 or ts) + 0.1):
+                continue
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                sm.append(float(f[2]))
+                smax.append(float(f[3]))
+                power.append(float(f[4]))
+            except ValueError:
+                continue
+            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
+                                 f[6:10]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        med = sorted(sm)[len(sm) // 2] if sm else None
+        return {"sm_mhz": med, "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+class Layer:
+    """One layer's resident state: KV cache, block summary, label slab, query."""
+
+    def __init__(self, T, w, shape, K, V, seq_lens, label, q, dev):
+        import torch
+
+        self.K = K.clone()
+        self.V = V.clone() if V is not None else None
+        self.q = q
+        edt = torch.int16 if w.dtype == 1 else torch.float32
+        self.meta = torch.empty((w.batch, w.n_kv_heads, w.n_blocks, 2, w.d_qk), dtype=edt, device=dev)
+        self.slab = torch.empty((w.batch, w.n_kv_heads, w.ctx, w.n_label), dtype=edt, device=dev)
+        T.tls_build_block_meta(shape, self.K, seq_lens, label, self.meta, self.slab)
+
+
+def gpu_arm(args, rank, world, local_rank):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    from two_level_sparse_quest_b200 import build as tls_build
+
+    tls_build.build()
+    from two_level_sparse_quest_b200 import tls as T
+    from two_level_sparse_quest_b200 import workloads as W
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    base = W.WORKLOADS[args.workload]
+    w = base.with_(seed=base.seed + 7919 * rank)  # each rank: its own sequences
+    shape = T.shape_from_workload(w)
+    inp = W.make_decode_inputs(w)
+    qs = W.make_query_stream(w.with_(ar_rho=0.5), steps=N_LAYERS)
+
+    def up(a):
+        return torch.from_numpy(np.ascontiguousarray(a.view(np.int16) if a.dtype == np.uint16 else a)).to(dev)
+
+    K0 = up(inp.K)
+    V0 = up(inp.V) if inp.V is not None else None
+    del inp.K
+    seq_lens, label = up(inp.seq_lens), up(inp.label_idx)
+    layers = [Layer(T, w, shape, K0, V0, seq_lens, label, up(qs[i]), dev) for i in range(N_LAYERS)]
+    del K0, V0
+    G = w.batch * w.n_kv_heads
+    ws = torch.zeros(T.tls_workspace_size(shape), dtype=torch.uint8, device=dev)
+    bidx = torch.empty((G, w.k_b), dtype=torch.int32, device=dev)
+    tidx = torch.empty((G, w.k_t), dtype=torch.int32, device=dev)
+    out = torch.empty((w.batch, w.n_q_heads, w.d_v), dtype=torch.float32, device=dev)
+    lse = torch.empty((w.batch, w.n_q_heads), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+
+    def step(L, ev=None):
+        if ev:
+            ev[0].record(stream)
+        T.tls_block_score_topk(shape, L.q, L.meta, seq_lens, bidx, None, ws, sh)
+        if ev:
+            ev[1].record(stream)
+        T.tls_token_score_topk(shape, L.q, L.slab, label, bidx, seq_lens, tidx, None, ws, sh)
+        if ev:
+            ev[2].record(stream)
+        T.tls_sparse_attn_decode(shape, L.q, L.K, L.V, tidx, out, lse, ws, sh)
+        if ev:
+            ev[3].record(stream)
+
+    launches_per_step = 5  # block score, block top-k, token score+top-k, attention split, merge
+    for i in range(args.warmup):
+        step(layers[i % N_LAYERS])
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, per-stage CUDA events on the launching stream
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[0])
+                           if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local_rank)
+    if rank == 0:
+        sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.mark("t0")
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(layers[i % N_LAYERS], evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    sampler.mark("t1")
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if rank == 0 else None
+    ms = t_start.elapsed_time(t_end)
+    st = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])] for e in evs])
+    stage_ms = st.mean(axis=0)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # ---- end to end through the C ABI with host buffers: H2D q, step, D2H out + lse
+    n_e2e = min(args.steps, 500)
+    q_host = [torch.empty(L.q.shape, dtype=L.q.dtype, pin_memory=True) for L in layers]
+    for i, L in enumerate(layers):
+        q_host[i].copy_(L.q.cpu())
+    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    lse_host = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    for i in range(3):
+        L = layers[i % N_LAYERS]
+        L.q.copy_(q_host[i % N_LAYERS], non_blocking=True)
+        step(L)
+        out_host.copy_(out, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(n_e2e):
+        L = layers[i % N_LAYERS]
+        L.q.copy_(q_host[i % N_LAYERS], non_blocking=True)
+        step(L)
+        out_host.copy_(out, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = layers[0].q.numel() * layers[0].q.element_size()
+    d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
+
+    if rank != 0:
+        return None
+    ab = algorithmic_bytes(w)
+    peaks = read_peaks()
+    step_ms = ms / args.steps
+    names = ["stage_block", "stage_token", "stage_attn"]
+    dom = int(np.argmax(stage_ms))
+    dom_bytes = ab[names[dom]]
+    achieved = dom_bytes / (stage_ms[dom] * 1e-3) / 1e9
+    res = {
+        "metric": METRIC,
+        "value": world * args.steps / (ms * 1e-3),
+        "unit": "steps/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == 1 else "f32",
+        "data": "synthetic: seeded Gaussian K/V with outlier channels and planted needle keys",
+        "config": {
+            "workload": args.workload, "batch": w.batch, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
+            "d_qk": w.d_qk, "d_v": w.d_v, "ctx": w.ctx, "block_size": w.block_size, "k_b": w.k_b, "k_t": w.k_t,
+            "n_label": w.n_label, "out_dtype": "f32",
+            "l2": f"inputs larger than L2: {N_LAYERS} layer copies rotated, {N_LAYERS * ab['total'] / 1e6:.0f} MB "
+                  f"of algorithmic bytes per rotation (L2 126 MB)",
+            "algorithmic_bytes_per_step": ab["total"],
+        },
+        "hbm_gbs": ab["total"] / (step_ms * 1e-3) / 1e9,
+        "hbm_frac_of_measured": ab["total"] / (step_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+        "hbm_frac_of_8000": ab["total"] / (step_ms * 1e-3) / 1e9 / 8000.0,
+        "stages_us": {n: float(v * 1e3) for n, v in zip(names, stage_ms)},
+        "roofline": {
+            "kernel": names[dom], "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
+            "traffic": read_traffic(names[dom]), "algorithmic_bytes_per_launch": dom_bytes,
+        },
+        "e2e": {"value": world * n_e2e / (e2e_ms * 1e-3), "unit": "steps/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": n_e2e},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+    }
+    return res
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample(args, budget_s: float):
+    """The fp64 oracle (single thread) on a bounded sample of the workload: the
+    step for a subset of the batch rows, scaled to a whole step."""
+    import numpy as np
+
+    from oracle import oracle as O
+    from two_level_sparse_quest_b200 import workloads as W
+
+    w = W.WORKLOADS[args.workload]
+    rows = 1
+    ws = w.with_(batch=rows)
+    inp = W.make_decode_inputs(ws)
+    s = O.shape_of(ws)
+    meta = O.build_meta(s, inp.K, inp.seq_lens)
+    times = []
+    t_all = time.time()
+    while True:
+        t0 = time.perf_counter()
+        O.decode_step(s, inp.q, inp.K, inp.V, meta, inp.seq_lens, inp.label_idx)
+        times.append(time.perf_counter() - t0)
+        if time.time() - t_all > budget_s or len(times) >= 20:
+            break
+    per_row = float(np.median(times)) / rows
+    per_step = per_row * w.batch
+    return {
+        "value": 1.0 / per_step, "unit": "steps/s", "cores": 1, "kind": "oracle",
+        "sample": f"{len(times)} run(s) of {rows} of {w.batch} batch rows (all {w.n_kv_heads} KV heads), "
+                  f"stages 1-5, fp64, single thread; scaled x{w.batch // rows} to one step",
+        "seconds_per_step": per_step,
+    }
+
+
+def reference_arm(args, rank, world):
+    if rank != 0:
+        return None
+    from two_level_sparse_quest_b200 import workloads as W
+
+    w = W.WORKLOADS[args.workload]
+    # warm-up and timed steps are each a bounded sample (one batch row)
+    cb = oracle_sample(args, budget_s=max(5.0, 3.0 * (args.steps + args.warmup)))
+    return {
+        "metric": METRIC, "impl": "reference", "value": cb["value"], "unit": "steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": cb["seconds_per_step"] * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic: seeded Gaussian K/V with outlier channels and planted needle keys",
+        "config": {"workload": args.workload, "batch": w.batch, "ctx": w.ctx, "k_b": w.k_b, "k_t": w.k_t},
+        "cpu_baseline": cb,
+        "e2e": {"value": cb["value"], "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "note": "reference arm = the fp64 CPU oracle (no runnable reference implementation exists)",
+    }
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="gqa96k_b8_bf16")
+    ap.add_argument("--impl", default="tls", choices=["tls", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = reference_arm(args, rank, world)
+        if res:
+            print(json.dumps(res), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    res = gpu_arm(args, rank, world, local_rank)
+    if rank == 0 and res is not None:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = oracle_sample(args, budget_s=15.0)
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,283 @@
+"""Shared helpers of the GPU parity tests: run the CUDA stages through the C ABI,
+run the oracle on the same seeded inputs, and compare with the rules below.
+
+Comparison rules (north star of this library):
+  * block summary and label slab: bit-exact (they are min / max / copies of
+    stored values);
+  * index sets (blocks, tokens): bit-exact, except swaps at the K-th boundary
+    whose two oracle fp64 scores differ by less than 1e-4 relative; swaps are
+    counted and reported;
+  * fp32 scores: within a bound derived from fp32 rounding of the kernel's
+    summation (block_score_bound, token_score_bound);
+  * attention output and lse: |gpu - oracle| <= 2e-3 + 2e-3 |oracle|.
+Inputs flow oracle -> GPU only (the oracle's selections may be fed to the next
+GPU stage to test it alone); no oracle input comes from the GPU.
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+import torch
+
+from oracle import oracle as O
+from two_level_sparse_quest_b200 import workloads as W
+
+U32 = 2.0 ** -24  # unit roundoff of fp32
+ATOL = 2e-3
+RTOL = 2e-3
+SWAP_RTOL = 1e-4
+
+REPORT = os.environ.get("TLS_PARITY_REPORT")
+
+
+def report(name: str, **kv):
+    if not REPORT:
+        return
+    os.makedirs(os.path.dirname(REPORT) or ".", exist_ok=True)
+    with open(REPORT, "a") as f:
+        f.write(json.dumps({"case": name, **kv}) + "\n")
+
+
+def tls():
+    from two_level_sparse_quest_b200 import tls as T
+
+    return T
+
+
+def to_dev(a: np.ndarray) -> torch.Tensor:
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def from_dev_elems(t: torch.Tensor, dtype: int) -> np.ndarray:
+    a = t.cpu().numpy()
+    return W.to_f64(a.view(np.uint16) if dtype == W.BF16 else a, dtype)
+
+
+class GpuInputs:
+    """Device copies of one decode step's inputs, plus the built summary and slab."""
+
+    def __init__(self, w: W.Workload, inp: W.DecodeInputs, out_dtype=0):
+        T = tls()
+        self.w, self.inp = w, inp
+        self.shape = T.shape_from_workload(w, out_dtype=out_dtype)
+        self.q = to_dev(inp.q)
+        self.K = to_dev(inp.K)
+        self.V = to_dev(inp.V) if inp.V is not None else None
+        self.seq_lens = to_dev(inp.seq_lens)
+        self.label = to_dev(inp.label_idx)
+        edt = torch.int16 if w.dtype == W.BF16 else torch.float32
+        B, H, nb, d = w.batch, w.n_kv_heads, w.n_blocks, w.d_qk
+        self.meta = torch.zeros((B, H, nb, 2, d), dtype=edt, device="cuda")
+        self.slab = torch.zeros((B, H, w.ctx, w.n_label), dtype=edt, device="cuda")
+        T.tls_build_block_meta(self.shape, self.K, self.seq_lens, self.label, self.meta, self.slab)
+        self.ws = torch.zeros(T.tls_workspace_size(self.shape), dtype=torch.uint8, device="cuda")
+
+    def block_stage(self, with_scores=True):
+        T, w = tls(), self.w
+        bidx = torch.full((w.batch, w.n_kv_heads, w.k_b), -7, dtype=torch.int32, device="cuda")
+        sc = torch.zeros((w.batch, w.n_kv_heads, w.n_blocks), dtype=torch.float32, device="cuda") if with_scores else None
+        T.tls_block_score_topk(self.shape, self.q, self.meta, self.seq_lens, bidx, sc, self.ws)
+        return bidx, sc
+
+    def token_stage(self, block_idx: torch.Tensor, with_scores=True):
+        T, w = tls(), self.w
+        tidx = torch.full((w.batch, w.n_kv_heads, w.k_t), -7, dtype=torch.int32, device="cuda")
+        C = w.k_b * w.block_size
+        sc = torch.zeros((w.batch, w.n_kv_heads, C), dtype=torch.float32, device="cuda") if with_scores else None
+        T.tls_token_score_topk(self.shape, self.q, self.slab, self.label, block_idx, self.seq_lens, tidx, sc, self.ws)
+        return tidx, sc
+
+    def attention(self, token_idx: torch.Tensor):
+        T, w = tls(), self.w
+        odt = torch.int16 if self.shape.out_dtype == W.BF16 else torch.float32
+        out = torch.zeros((w.batch, w.n_q_heads, w.d_v), dtype=odt, device="cuda")
+        lse = torch.zeros((w.batch, w.n_q_heads), dtype=torch.float32, device="cuda")
+        T.tls_sparse_attn_decode(self.shape, self.q, self.K, self.V, token_idx, out, lse, self.ws)
+        return out, lse
+
+    def out_f64(self, out: torch.Tensor) -> np.ndarray:
+        return from_dev_elems(out, self.shape.out_dtype)
+
+
+class OracleRun:
+    """The oracle's own chain on the same inputs."""
+
+    def __init__(self, w: W.Workload, inp: W.DecodeInputs):
+        s = O.shape_of(w)
+        self.s = s
+        self.meta = O.build_meta(s, inp.K, inp.seq_lens)
+        self.block_scores = O.block_scores(s, inp.q, self.meta, inp.seq_lens)
+        self.block_idx = O.select_blocks(s, self.block_scores, inp.seq_lens)
+        self.cand_scores, self.cand_tok = O.token_scores(s, inp.q, inp.K, inp.label_idx, self.block_idx, inp.seq_lens)
+        self.token_idx = O.select_tokens(s, self.cand_scores, self.cand_tok)
+        self.out, self.lse = O.attention(s, inp.q, inp.K, inp.V, self.token_idx)
+
+
+# ---------------------------------------------------------------- comparisons
+def check_meta(w, inp, gpu: GpuInputs, orc: OracleRun):
+    gm = from_dev_elems(gpu.meta, w.dtype)
+    for b in range(w.batch):
+        nb = -(-int(inp.seq_lens[b]) // w.block_size)
+        np.testing.assert_array_equal(gm[b, :, :nb], orc.meta[b, :, :nb])
+    # the slab is a copy of stored values: compare the stored bits
+    gs = gpu.slab.cpu().numpy()
+    gs = gs.view(np.uint16) if w.dtype == W.BF16 else gs.view(np.uint32)
+    Kr = inp.K.view(np.uint16) if w.dtype == W.BF16 else inp.K.view(np.uint32)
+    for b in range(w.batch):
+        L = int(inp.seq_lens[b])
+        np.testing.assert_array_equal(gs[b, :, :L], Kr[b, :, :L][..., inp.label_idx])
+
+
+def block_score_bound(w, inp, orc: OracleRun) -> np.ndarray:
+    """fp32 rounding bound of the kernel's block score: the head sum folded into
+    Q+/Q- (G terms) and a 2d-term dot, each term bounded by |q| max(|M|,|m|)."""
+    q = W.to_f64(inp.q, w.dtype).reshape(w.batch, w.n_kv_heads, w.group, w.d_qk)
+    A = np.abs(q).sum(axis=2)  # [B][H][d]
+    mag = np.maximum(np.abs(orc.meta[:, :, :, 0]), np.abs(orc.meta[:, :, :, 1]))  # [B][H][nb][d]
+    mag = np.nan_to_num(mag)
+    return 2.0 * (2 * w.d_qk + w.group + 2) * U32 * np.einsum("bhd,bhnd->bhn", A, mag)
+
+
+def token_score_bound(w, inp, orc: OracleRun, block_idx: np.ndarray) -> np.ndarray:
+    """fp32 rounding bound of the kernel's token score: Qbar_L = sum of G heads,
+    then an r-term dot; each term bounded by |q_{h,c}| |K[t,c]|."""
+    q = W.to_f64(inp.q, w.dtype).reshape(w.batch, w.n_kv_heads, w.group, w.d_qk)[..., inp.label_idx]
+    C = w.k_b * w.block_size
+    out = np.zeros((w.batch, w.n_kv_heads, C))
+    j = np.arange(C)
+    for b in range(w.batch):
+        for g in range(w.n_kv_heads):
+            blk = block_idx[b, g][j // w.block_size]
+            t = blk * w.block_size + j % w.block_size
+            ok = (blk >= 0) & (t < inp.seq_lens[b])
+            rows = inp.K[b, g][np.where(ok, t, 0)][:, inp.label_idx]
+            kk = np.abs(W.to_f64(rows, w.dtype))
+            out[b, g] = np.where(ok, kk @ np.abs(q[b, g]).sum(axis=0), 0.0)
+    return 2.0 * (w.n_label + w.group + 2) * U32 * out
+
+
+def check_scores(gpu_scores: np.ndarray, ora_scores: np.ndarray, bound: np.ndarray, what: str):
+    g = gpu_scores.astype(np.float64)
+    o = ora_scores
+    inval = np.isneginf(o)
+    assert (np.isneginf(g) == inval).all(), f"{what}: invalid-entry pattern differs"
+    err = np.abs(g[~inval] - o[~inval])
+    lim = bound[~inval] + 1e-30
+    bad = err > lim
+    assert not bad.any(), f"{what}: {bad.sum()} scores outside the fp32 bound; worst {err.max():.3e}"
+
+
+def check_selection(gpu_ids: np.ndarray, ids: np.ndarray, scores: np.ndarray, k: int, what: str) -> int:
+    """gpu_ids: kernel output (ascending, -1 padded).  ids/scores: the oracle's
+    candidate ids and fp64 scores.  Returns the number of boundary swaps."""
+    sel = gpu_ids[gpu_ids >= 0]
+    m = min(k, len(ids))
+    assert len(sel) == m, f"{what}: {len(sel)} selected, expected {m}"
+    assert (gpu_ids[m:] == -1).all(), f"{what}: padding"
+    assert (np.diff(sel) > 0).all(), f"{what}: not strictly ascending"
+    want, _ = O.topk(scores, k, ids=ids, out_cap=k)
+    want = want[want >= 0]
+    A, B = set(sel.tolist()), set(want.tolist())
+    if A == B:
+        return 0
+    sc = dict(zip(ids.tolist(), scores.tolist()))
+    assert A <= set(sc), f"{what}: selected ids that are not candidates"
+    s_in = [sc[x] for x in A - B]     # selected by the GPU only
+    s_out = [sc[y] for y in B - A]    # selected by the oracle only
+    hi, lo = max(s_out), min(s_in)
+    assert hi - lo <= SWAP_RTOL * max(abs(hi), abs(lo)), f"{what}: swap beyond 1e-4 relative ({hi} vs {lo})"
+    return len(A - B)
+
+
+def check_selection_self_consistent(gpu_ids: np.ndarray, cand_ids: np.ndarray, gpu_scores: np.ndarray, what: str):
+    """Property of a correct top-k on the kernel's own fp32 scores: every kept
+    score >= every dropped score, and among equal scores at the boundary the
+    kept ids are the lower ones."""
+    sel = set(gpu_ids[gpu_ids >= 0].tolist())
+    if not sel:
+        return
+    keep = np.array([c in sel for c in cand_ids.tolist()])
+    s = gpu_scores.astype(np.float32)
+    if keep.all() or not keep.any():
+        return
+    kmin = s[keep].min()
+    dmax = s[~keep].max()
+    assert kmin >= dmax, f"{what}: kept score {kmin} < dropped score {dmax}"
+    if kmin == dmax:
+        kept_eq = cand_ids[keep & (s == kmin)]
+        drop_eq = cand_ids[~keep & (s == kmin)]
+        assert kept_eq.max() < drop_eq.min(), f"{what}: tie not broken toward the lower id"
+
+
+def check_attention(gout: np.ndarray, glse: np.ndarray, oout: np.ndarray, olse: np.ndarray, what: str):
+    err = np.abs(gout - oout)
+    lim = ATOL + RTOL * np.abs(oout)
+    assert (err <= lim).all(), f"{what}: out error {err.max():.3e} ({(err > lim).sum()} elements)"
+    inf = np.isneginf(olse)
+    assert (np.isneginf(glse) == inf).all(), f"{what}: lse -inf pattern"
+    e2 = np.abs(glse[~inf] - olse[~inf])
+    assert (e2 <= ATOL + RTOL * np.abs(olse[~inf])).all(), f"{what}: lse error {e2.max() if e2.size else 0:.3e}"
+    return float(err.max()) if err.size else 0.0
+
+
+def full_stage_parity(w: W.Workload, seq_lens=None, out_dtype=0, name=None):
+    """Every stage against the oracle on one seeded input; returns a summary dict."""
+    name = name or w.name
+    inp = W.make_decode_inputs(w, seq_lens=seq_lens)
+    orc = OracleRun(w, inp)
+    gpu = GpuInputs(w, inp, out_dtype=out_dtype)
+    check_meta(w, inp, gpu, orc)
+    # stage 1+2
+    bidx, bsc = gpu.block_stage()
+    torch.cuda.synchronize()
+    bidx, bsc = bidx.cpu().numpy(), bsc.cpu().numpy()
+    check_scores(bsc, orc.block_scores, block_score_bound(w, inp, orc), f"{name} block scores")
+    swaps_b = 0
+    for b in range(w.batch):
+        nb = -(-int(inp.seq_lens[b]) // w.block_size)
+        ids = np.arange(nb, dtype=np.int32)
+        for g in range(w.n_kv_heads):
+            swaps_b += check_selection(bidx[b, g], ids, orc.block_scores[b, g, :nb], w.k_b, f"{name} blocks b{b} g{g}")
+            check_selection_self_consistent(bidx[b, g], ids, bsc[b, g, :nb], f"{name} blocks b{b} g{g}")
+    # stage 3+4 on the oracle's block selection
+    tidx, tsc = gpu.token_stage(to_dev(orc.block_idx))
+    torch.cuda.synchronize()
+    tidx, tsc = tidx.cpu().numpy(), tsc.cpu().numpy()
+    check_scores(tsc, orc.cand_scores, token_score_bound(w, inp, orc, orc.block_idx), f"{name} token scores")
+    swaps_t = 0
+    for b in range(w.batch):
+        for g in range(w.n_kv_heads):
+            ok = orc.cand_tok[b, g] >= 0
+            ids = orc.cand_tok[b, g][ok]
+            swaps_t += check_selection(tidx[b, g], ids, orc.cand_scores[b, g][ok], w.k_t, f"{name} tokens b{b} g{g}")
+            check_selection_self_consistent(tidx[b, g], ids, tsc[b, g][ok], f"{name} tokens b{b} g{g}")
+    # stage 5 on the oracle's token selection
+    out, lse = gpu.attention(to_dev(orc.token_idx))
+    torch.cuda.synchronize()
+    err = check_attention(gpu.out_f64(out), lse.cpu().numpy().astype(np.float64), orc.out, orc.lse, f"{name} attention")
+    # chained: the GPU's own selections all the way
+    cb, _ = gpu.block_stage(with_scores=False)
+    ct, _ = gpu.token_stage(cb, with_scores=False)
+    cout, clse = gpu.attention(ct)
+    torch.cuda.synchronize()
+    cb, ct = cb.cpu().numpy(), ct.cpu().numpy()
+    cout, clse = gpu.out_f64(cout), clse.cpu().numpy().astype(np.float64)
+    np.testing.assert_array_equal(cb, bidx)  # deterministic
+    same_groups = 0
+    G = w.group
+    for b in range(w.batch):
+        for g in range(w.n_kv_heads):
+            if (cb[b, g] == orc.block_idx[b, g]).all():
+                np.testing.assert_array_equal(ct[b, g], tidx[b, g])
+            if (ct[b, g] == orc.token_idx[b, g]).all():
+                same_groups += 1
+                hs = slice(g * G, (g + 1) * G)
+                check_attention(cout[b, hs], clse[b, hs], orc.out[b, hs], orc.lse[b, hs], f"{name} chained b{b} g{g}")
+    res = dict(block_swaps=swaps_b, token_swaps=swaps_t, attn_max_abs_err=err,
+               chained_groups_identical=same_groups, groups=w.batch * w.n_kv_heads)
+    report(name, **res)
+    return res

@@ -1,0 +1,78 @@
+"""GPU parity: every stage of the CUDA path against the fp64 oracle (B200).
+
+Small cases span several tiles and ragged tails and cover the edge cases
+(ragged and empty sequences, partial last blocks, k_b >= number of blocks,
+k_t >= candidates, group sizes 1/2/4/8, bf16 output).  The five named
+workloads run at their full sizes, in the launch configuration the benchmark
+uses.  Comparison rules are in tests/_parity.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+from two_level_sparse_quest_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.fail("CUDA device required for -m gpu tests")
+    from two_level_sparse_quest_b200 import build
+
+    build.build()
+
+
+def P():
+    from tests import _parity
+
+    return _parity
+
+
+SMALL = {
+    "tiny_f32_ragged": (W.WORKLOADS["tiny_gqa4k_f32"].with_(batch=3, ctx=1000, k_b=8, k_t=100), [1000, 777, 33]),
+    "gqa_bf16_small": (W.WORKLOADS["gqa48k_bf16"].with_(batch=2, ctx=4096, k_b=24, k_t=300), [4096, 4001]),
+    "gqa_bf16_g8": (W.WORKLOADS["gqa48k_bf16"].with_(n_q_heads=64, ctx=2048, k_b=16, k_t=257), None),
+    "gqa_bf16_g1": (W.WORKLOADS["gqa48k_bf16"].with_(n_q_heads=8, ctx=2048, k_b=16, k_t=130), None),
+    "gqa_bf16_g2_d64": (W.WORKLOADS["gqa48k_bf16"].with_(n_q_heads=16, d_qk=64, d_v=64, ctx=3000, k_b=20,
+                                                        k_t=200, n_outlier=4), None),
+    "gqa_f32_d128": (W.WORKLOADS["tiny_gqa4k_f32"].with_(batch=2, d_qk=128, d_v=128, n_kv_heads=2, n_q_heads=8, ctx=2500,
+                                                         k_b=10, k_t=96), [2500, 1501]),
+    "clamp_kb_ge_nblocks": (W.WORKLOADS["gqa48k_bf16"].with_(ctx=200, k_b=64, k_t=50), [200]),
+    "clamp_kt_ge_candidates": (W.WORKLOADS["gqa48k_bf16"].with_(ctx=1024, k_b=4, k_t=500), [1024]),
+    "empty_and_tiny_sequences": (W.WORKLOADS["tiny_gqa4k_f32"].with_(batch=4, ctx=512, k_b=4, k_t=40),
+                                 [0, 1, 31, 512]),
+    "block_size_16_odd_ctx": (W.WORKLOADS["gqa48k_bf16"].with_(block_size=16, ctx=1999, k_b=40, k_t=333), None),
+    "mla_small": (W.WORKLOADS["mla64k_b4_bf16"].with_(batch=2, ctx=4096, k_b=16, k_t=300, n_needles=4),
+                  [4096, 3000]),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_small_parity(name):
+    w, sl = SMALL[name]
+    res = P().full_stage_parity(w, seq_lens=sl, name=name)
+    assert res["chained_groups_identical"] >= 0
+
+
+def test_bf16_output_parity():
+    w = W.WORKLOADS["gqa48k_bf16"].with_(ctx=4096, k_b=24, k_t=300)
+    P().full_stage_parity(w, out_dtype=W.BF16, name="bf16_out")
+
+
+def test_full_selection_equals_full_attention_gpu():
+    # K_b = all blocks, K_t = all tokens: the sparse step is dense attention
+    w = W.WORKLOADS["gqa48k_bf16"].with_(ctx=2048, k_b=64, k_t=2048)
+    P().full_stage_parity(w, name="full_selection")
+
+
+FULL = ["tiny_gqa4k_f32", "gqa48k_bf16", "gqa96k_b8_bf16", "mla64k_b4_bf16"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_size_parity(name):
+    res = P().full_stage_parity(W.WORKLOADS[name], name=f"full:{name}")
+    # spec: index sets bit-exact except counted boundary swaps
+    assert res["block_swaps"] <= max(1, res["groups"] // 8)
+    assert res["token_swaps"] <= max(1, res["groups"] // 8)

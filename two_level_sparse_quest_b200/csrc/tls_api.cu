@@ -1,0 +1,362 @@
+// tls_api.cu -- the extern "C" entry points of libtls.so (declared in
+// include/tls.h): host-side argument checks, workspace layout, kernel
+// dispatch and error reporting.  Nothing here computes; every step of the
+// decode path runs in the kernels of tls_meta.cu, tls_select.cu, tls_attn.cu
+// and tls_offload.cu.
+#include <cuda_runtime.h>
+
+#include <chrono>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <thread>
+
+#include "tls.h"
+#include "tls_internal.h"
+
+namespace {
+
+thread_local std::string g_err;
+
+tls_status fail(tls_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+tls_status fail(tls_status st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+
+tls_status cuda_status(cudaError_t e, const char *what) {
+  if (e == cudaSuccess) return TLS_OK;
+  return fail(TLS_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int elt_bytes(const tls_shape *s) { return s->kv_dtype == TLS_BF16 ? 2 : 4; }
+int n_blocks_max(const tls_shape *s) { return (s->max_ctx + s->block_size - 1) / s->block_size; }
+
+int device_sms() {
+  static int cache[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    cache[dev] = v;
+  }
+  return cache[dev];
+}
+
+// Common shape checks.  `need_attn` adds the attention kernel-set checks.
+tls_status check_shape(const tls_shape *s) {
+  if (!s) return fail(TLS_ERR_INVALID_ARG, "shape is NULL");
+  if (s->batch < 0) return fail(TLS_ERR_INVALID_ARG, "batch < 0");
+  if (s->n_kv_heads < 1 || s->n_q_heads < 1 || s->n_q_heads % s->n_kv_heads)
+    return fail(TLS_ERR_INVALID_ARG, "n_q_heads (%d) must be a positive multiple of n_kv_heads (%d)", s->n_q_heads,
+                s->n_kv_heads);
+  if (s->kv_dtype != TLS_F32 && s->kv_dtype != TLS_BF16) return fail(TLS_ERR_INVALID_ARG, "kv_dtype %d", s->kv_dtype);
+  if (s->out_dtype != TLS_F32 && s->out_dtype != TLS_BF16) return fail(TLS_ERR_INVALID_ARG, "out_dtype %d", s->out_dtype);
+  if (s->block_size < 1) return fail(TLS_ERR_INVALID_ARG, "block_size < 1");
+  if (s->max_ctx < 1) return fail(TLS_ERR_INVALID_ARG, "max_ctx < 1");
+  if (s->k_b < 1 || s->k_t < 1) return fail(TLS_ERR_INVALID_ARG, "k_b and k_t must be >= 1");
+  if (s->d_qk < 1 || s->d_v < 1) return fail(TLS_ERR_INVALID_ARG, "d_qk and d_v must be >= 1");
+  if (s->v_is_k_prefix && s->d_v > s->d_qk) return fail(TLS_ERR_INVALID_ARG, "v_is_k_prefix needs d_v <= d_qk");
+  if (static_cast<long long>(s->batch) * s->n_kv_heads > 65535)
+    return fail(TLS_ERR_UNSUPPORTED, "batch * n_kv_heads > 65535");
+  const int G = s->n_q_heads / s->n_kv_heads;
+  if (s->v_is_k_prefix) {
+    if (s->kv_dtype != TLS_BF16 || s->d_qk != 576 || s->d_v != 512 || G % 4 || G > 128)
+      return fail(TLS_ERR_UNSUPPORTED, "latent attention supports bf16, d_qk 576, d_v 512, G a multiple of 4 <= 128");
+  } else {
+    if (s->d_qk != s->d_v || (s->d_qk != 64 && s->d_qk != 128))
+      return fail(TLS_ERR_UNSUPPORTED, "GQA supports d_qk = d_v in {64, 128} (got %d, %d)", s->d_qk, s->d_v);
+    if (G != 1 && G != 2 && G != 4 && G != 8) return fail(TLS_ERR_UNSUPPORTED, "GQA group size %d not in {1,2,4,8}", G);
+  }
+  if (n_blocks_max(s) > tls::kMaxSelectKeys)
+    return fail(TLS_ERR_UNSUPPORTED, "ceil(max_ctx / block_size) = %d > %d", n_blocks_max(s), tls::kMaxSelectKeys);
+  if (s->k_b > 1024) return fail(TLS_ERR_UNSUPPORTED, "k_b %d > 1024", s->k_b);
+  if (static_cast<long long>(s->k_b) * s->block_size > tls::kMaxSelectKeys)
+    return fail(TLS_ERR_UNSUPPORTED, "k_b * block_size = %lld > %d", static_cast<long long>(s->k_b) * s->block_size,
+                tls::kMaxSelectKeys);
+  const bool r_ok = s->kv_dtype == TLS_BF16
+                        ? (s->n_label == 8 || s->n_label == 16 || s->n_label == 32 || s->n_label == 64)
+                        : (s->n_label == 4 || s->n_label == 8 || s->n_label == 16 || s->n_label == 32);
+  if (!r_ok) return fail(TLS_ERR_UNSUPPORTED, "n_label %d unsupported for this dtype", s->n_label);
+  if (s->n_label > s->d_qk) return fail(TLS_ERR_INVALID_ARG, "n_label > d_qk");
+  return TLS_OK;
+}
+
+#define CHECK_PTR(p, a)                                                                          \
+  do {                                                                                           \
+    if (!(p)) return fail(TLS_ERR_INVALID_ARG, "%s is NULL", #p);                                \
+    if (!aligned((p), (a))) return fail(TLS_ERR_INVALID_ARG, "%s is not %d-byte aligned", #p, a); \
+  } while (0)
+
+float scale_of(const tls_shape *s) {
+  return s->softmax_scale > 0.f ? s->softmax_scale : 1.0f / std::sqrt(static_cast<float>(s->d_qk));
+}
+
+tls::AttnArgs attn_args(const tls_shape *s) {
+  tls::AttnArgs a{};
+  a.batch = s->batch;
+  a.n_q_heads = s->n_q_heads;
+  a.n_kv_heads = s->n_kv_heads;
+  a.d_qk = s->d_qk;
+  a.d_v = s->d_v;
+  a.v_is_k_prefix = s->v_is_k_prefix;
+  a.block_size = s->block_size;
+  a.n_blocks_max = n_blocks_max(s);
+  a.max_ctx = s->max_ctx;
+  a.k_t = s->k_t;
+  a.dtype = s->kv_dtype;
+  a.out_dtype = s->out_dtype;
+  a.scale_log2 = scale_of(s) * 1.4426950408889634f;
+  a.num_sms = device_sms();
+  return a;
+}
+
+// Workspace layout: [block scores | attention partials], 256-byte aligned.
+struct WsLayout {
+  size_t scores_off, scores_bytes, part_off, part_bytes, total;
+};
+
+bool ws_layout(const tls_shape *s, bool paged, WsLayout *w) {
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  w->scores_off = 0;
+  w->scores_bytes = up(static_cast<size_t>(s->batch) * s->n_kv_heads * n_blocks_max(s) * sizeof(float));
+  tls::AttnArgs a = attn_args(s);
+  a.paged = paged;
+  tls::AttnPlan p;
+  if (!tls::attn_plan(a, &p)) return false;
+  w->part_off = w->scores_bytes;
+  w->part_bytes = up(p.part_floats * sizeof(float));
+  w->total = w->part_off + w->part_bytes;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *tls_version(void) { return "tls 0.1 sm_100a"; }
+
+const char *tls_last_error(void) { return g_err.c_str(); }
+
+size_t tls_workspace_size(const tls_shape *s) {
+  if (check_shape(s) != TLS_OK) return 0;
+  WsLayout w;
+  if (!ws_layout(s, false, &w)) {
+    fail(TLS_ERR_UNSUPPORTED, "no attention plan for this shape");
+    return 0;
+  }
+  WsLayout wp;
+  if (!s->v_is_k_prefix && ws_layout(s, true, &wp) && wp.total > w.total) return wp.total;
+  return w.total;
+}
+
+tls_status tls_build_block_meta(const tls_shape *s, const void *K, const int32_t *seq_lens, const int32_t *label_idx,
+                                void *meta_out, void *slab_out, void *stream) {
+  tls_status st = check_shape(s);
+  if (st != TLS_OK) return st;
+  if (s->batch == 0) return TLS_OK;
+  CHECK_PTR(K, 16);
+  CHECK_PTR(seq_lens, 4);
+  CHECK_PTR(meta_out, 16);
+  if (slab_out) {
+    CHECK_PTR(label_idx, 4);
+    CHECK_PTR(slab_out, 16);
+  }
+  tls::MetaArgs a{K, seq_lens, label_idx, meta_out, slab_out, s->batch, s->n_kv_heads, s->d_qk, s->block_size,
+                  n_blocks_max(s), s->max_ctx, s->n_label, s->kv_dtype};
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  st = cuda_status(tls::launch_build_meta(a, cs), "build_meta launch");
+  if (st != TLS_OK || !slab_out) return st;
+  return cuda_status(tls::launch_build_slab(a, cs), "build_slab launch");
+}
+
+tls_status tls_block_score_topk(const tls_shape *s, const void *q, const void *meta, const int32_t *seq_lens,
+                                int32_t *block_idx_out, float *block_score_out, void *ws, size_t ws_bytes,
+                                void *stream) {
+  tls_status st = check_shape(s);
+  if (st != TLS_OK) return st;
+  if (s->batch == 0) return TLS_OK;
+  CHECK_PTR(q, 16);
+  CHECK_PTR(meta, 16);
+  CHECK_PTR(seq_lens, 4);
+  CHECK_PTR(block_idx_out, 4);
+  if (block_score_out && !aligned(block_score_out, 4)) return fail(TLS_ERR_INVALID_ARG, "block_score_out misaligned");
+  float *scores = block_score_out;
+  if (!scores) {
+    WsLayout w;
+    if (!ws_layout(s, false, &w)) return fail(TLS_ERR_UNSUPPORTED, "no plan for this shape");
+    if (!ws || ws_bytes < w.scores_off + w.scores_bytes || !aligned(ws, 256))
+      return fail(TLS_ERR_WORKSPACE, "workspace too small or not 256-byte aligned (need %zu bytes)",
+                  w.scores_off + w.scores_bytes);
+    scores = reinterpret_cast<float *>(static_cast<char *>(ws) + w.scores_off);
+  }
+  tls::BlockScoreArgs a{q, meta, seq_lens, scores, block_idx_out, s->batch, s->n_q_heads, s->n_kv_heads, s->d_qk,
+                        s->block_size, n_blocks_max(s), s->max_ctx, s->k_b, s->kv_dtype, device_sms()};
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  st = cuda_status(tls::launch_block_score(a, cs), "block_score launch");
+  if (st != TLS_OK) return st;
+  return cuda_status(tls::launch_block_topk(a, cs), "block_topk launch");
+}
+
+tls_status tls_token_score_topk(const tls_shape *s, const void *q, const void *slab, const int32_t *label_idx,
+                                const int32_t *block_idx, const int32_t *seq_lens, int32_t *token_idx_out,
+                                float *token_score_out, void *ws, size_t ws_bytes, void *stream) {
+  (void)ws;
+  (void)ws_bytes;
+  tls_status st = check_shape(s);
+  if (st != TLS_OK) return st;
+  if (s->batch == 0) return TLS_OK;
+  CHECK_PTR(q, 16);
+  CHECK_PTR(slab, 16);
+  CHECK_PTR(label_idx, 4);
+  CHECK_PTR(block_idx, 4);
+  CHECK_PTR(seq_lens, 4);
+  CHECK_PTR(token_idx_out, 4);
+  if (token_score_out && !aligned(token_score_out, 4)) return fail(TLS_ERR_INVALID_ARG, "token_score_out misaligned");
+  tls::TokenArgs a{q, slab, label_idx, block_idx, seq_lens, token_idx_out, token_score_out, s->batch, s->n_q_heads,
+                   s->n_kv_heads, s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->n_label, s->k_b, s->k_t,
+                   s->kv_dtype};
+  return cuda_status(tls::launch_token_topk(a, static_cast<cudaStream_t>(stream)), "token_topk launch");
+}
+
+static tls_status attn_common(const tls_shape *s, const void *q, const void *K, const void *V,
+                              const int32_t *token_idx, const int32_t *slot_of_block, int32_t n_slots, void *out,
+                              float *lse_out, void *ws, size_t ws_bytes, void *stream, bool paged) {
+  tls_status st = check_shape(s);
+  if (st != TLS_OK) return st;
+  if (s->batch == 0) return TLS_OK;
+  CHECK_PTR(q, 16);
+  CHECK_PTR(K, 16);
+  if (!paged && !s->v_is_k_prefix) CHECK_PTR(V, 16);
+  CHECK_PTR(token_idx, 4);
+  CHECK_PTR(out, 16);
+  if (lse_out && !aligned(lse_out, 4)) return fail(TLS_ERR_INVALID_ARG, "lse_out misaligned");
+  if (paged) {
+    if (s->v_is_k_prefix) return fail(TLS_ERR_UNSUPPORTED, "the block cache holds GQA K/V blocks only");
+    CHECK_PTR(slot_of_block, 4);
+    if (n_slots < 1) return fail(TLS_ERR_INVALID_ARG, "n_slots < 1");
+  }
+  WsLayout w;
+  if (!ws_layout(s, paged, &w)) return fail(TLS_ERR_UNSUPPORTED, "no attention plan for this shape");
+  if (!ws || ws_bytes < w.total || !aligned(ws, 256))
+    return fail(TLS_ERR_WORKSPACE, "workspace too small or not 256-byte aligned (need %zu bytes)", w.total);
+  tls::AttnArgs a = attn_args(s);
+  a.q = q;
+  a.K = K;
+  a.V = V;
+  a.token_idx = token_idx;
+  a.slot_of_block = slot_of_block;
+  a.n_slots = n_slots;
+  a.out = out;
+  a.lse = lse_out;
+  a.part = reinterpret_cast<float *>(static_cast<char *>(ws) + w.part_off);
+  a.paged = paged;
+  tls::AttnPlan p;
+  if (!tls::attn_plan(a, &p)) return fail(TLS_ERR_UNSUPPORTED, "no attention plan for this shape");
+  return cuda_status(tls::launch_attention(a, p, static_cast<cudaStream_t>(stream)), "attention launch");
+}
+
+tls_status tls_sparse_attn_decode(const tls_shape *s, const void *q, const void *K, const void *V,
+                                  const int32_t *token_idx, void *out, float *lse_out, void *ws, size_t ws_bytes,
+                                  void *stream) {
+  return attn_common(s, q, K, V, token_idx, nullptr, 0, out, lse_out, ws, ws_bytes, stream, false);
+}
+
+tls_status tls_sparse_attn_decode_paged(const tls_shape *s, const void *q, const void *cache,
+                                        const int32_t *slot_of_block, int32_t n_slots, const int32_t *token_idx,
+                                        void *out, float *lse_out, void *ws, size_t ws_bytes, void *stream) {
+  return attn_common(s, q, cache, nullptr, token_idx, slot_of_block, n_slots, out, lse_out, ws, ws_bytes, stream,
+                     true);
+}
+
+static tls_status offload_check(const tls_shape *s, int32_t n_slots) {
+  tls_status st = check_shape(s);
+  if (st != TLS_OK) return st;
+  if (s->v_is_k_prefix) return fail(TLS_ERR_UNSUPPORTED, "the block cache holds GQA K/V blocks only");
+  if (n_slots < 1 || n_slots > 4096) return fail(TLS_ERR_INVALID_ARG, "n_slots %d not in [1, 4096]", n_slots);
+  return TLS_OK;
+}
+
+tls_status tls_offload_reset(const tls_shape *s, int32_t n_slots, int32_t *slot_of_block, int32_t *block_of_slot,
+                             void *stream) {
+  tls_status st = offload_check(s, n_slots);
+  if (st != TLS_OK) return st;
+  if (s->batch == 0) return TLS_OK;
+  CHECK_PTR(slot_of_block, 4);
+  CHECK_PTR(block_of_slot, 4);
+  tls::OffloadArgs a{};
+  a.slot_of_block = slot_of_block;
+  a.block_of_slot = block_of_slot;
+  a.batch = s->batch;
+  a.n_kv_heads = s->n_kv_heads;
+  a.n_blocks_max = n_blocks_max(s);
+  a.n_slots = n_slots;
+  return cuda_status(tls::launch_offload_reset(a, static_cast<cudaStream_t>(stream)), "offload_reset launch");
+}
+
+tls_status tls_prefetch_diff(const tls_shape *s, int32_t n_slots, const void *host_kv, void *cache,
+                             int32_t *slot_of_block, int32_t *block_of_slot, const int32_t *prev_block_idx,
+                             const int32_t *next_block_idx, int32_t *n_new_out, int32_t *jobs_ws, void *stream) {
+  tls_status st = offload_check(s, n_slots);
+  if (st != TLS_OK) return st;
+  if (s->batch == 0) return TLS_OK;
+  CHECK_PTR(host_kv, 16);
+  CHECK_PTR(cache, 16);
+  CHECK_PTR(slot_of_block, 4);
+  CHECK_PTR(block_of_slot, 4);
+  CHECK_PTR(next_block_idx, 4);
+  CHECK_PTR(n_new_out, 4);
+  CHECK_PTR(jobs_ws, 4);
+  if (prev_block_idx && !aligned(prev_block_idx, 4)) return fail(TLS_ERR_INVALID_ARG, "prev_block_idx misaligned");
+  void *dev_host = nullptr;
+  cudaError_t e = cudaHostGetDevicePointer(&dev_host, const_cast<void *>(host_kv), 0);
+  if (e != cudaSuccess || !dev_host) {
+    cudaGetLastError();  // clear the error this query recorded
+    return fail(TLS_ERR_INVALID_ARG, "host_kv is not page-locked host memory visible to the device");
+  }
+  tls::OffloadArgs a{};
+  a.host_kv = dev_host;
+  a.cache = cache;
+  a.slot_of_block = slot_of_block;
+  a.block_of_slot = block_of_slot;
+  a.prev_block_idx = prev_block_idx;
+  a.next_block_idx = next_block_idx;
+  a.n_new = n_new_out;
+  a.jobs = jobs_ws;
+  a.batch = s->batch;
+  a.n_kv_heads = s->n_kv_heads;
+  a.d = s->d_qk;
+  a.block_size = s->block_size;
+  a.n_blocks_max = n_blocks_max(s);
+  a.k_b = s->k_b;
+  a.n_slots = n_slots;
+  a.dtype = s->kv_dtype;
+  return cuda_status(tls::launch_prefetch_diff(a, static_cast<cudaStream_t>(stream)), "prefetch_diff launch");
+}
+
+tls_status tls_wait_event(void *event, int32_t timeout_ms) {
+  if (!event) return fail(TLS_ERR_INVALID_ARG, "event is NULL");
+  if (timeout_ms < 0) timeout_ms = 0;
+  const auto t0 = std::chrono::steady_clock::now();
+  for (;;) {
+    cudaError_t e = cudaEventQuery(static_cast<cudaEvent_t>(event));
+    if (e == cudaSuccess) return TLS_OK;
+    if (e != cudaErrorNotReady) return cuda_status(e, "event query");
+    const auto ms =
+        std::chrono::duration_cast<std::chrono::milliseconds>(std::chrono::steady_clock::now() - t0).count();
+    if (ms >= timeout_ms) return fail(TLS_ERR_TIMEOUT, "event not complete after %d ms", timeout_ms);
+    std::this_thread::sleep_for(std::chrono::microseconds(200));
+  }
+}
+
+}  // extern "C"

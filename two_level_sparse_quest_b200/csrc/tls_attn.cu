@@ -1,0 +1,400 @@
+// tls_attn.cu -- stage 5 of the AsyncTLS decode step: exact softmax attention
+// over the gathered K/V rows of the selected tokens (gist.science (es) section
+// 2.A.2: the final attention runs at token precision on the K_t kept tokens).
+//
+// Design (B200):
+//  * Work = (unit, tile): a unit is one KV group (all G heads of a GQA group, or
+//    a chunk of HG heads of a latent group); a tile is 32 selected tokens.  The
+//    flattened tile space is cut into equal contiguous ranges, one per warp of a
+//    persistent grid (one CTA per SM), so every warp streams the same number of
+//    gathered rows and never waits on another warp.
+//  * Each warp runs its own NS-stage cp.async pipeline: row offsets of the
+//    tile's tokens go to shared memory, then the warp gathers the 32 K rows
+//    (and V rows) as 16-byte async copies (zero-fill for masked tokens) into a
+//    private stage buffer.  K rows are stored with their 16-byte chunks XOR-
+//    swizzled by (row & 7) so that lane r reading row r is conflict-free.
+//  * QK: lane r owns token r of the tile and dots its K row with the group's
+//    queries (fp32 in shared memory, pre-scaled by tau * log2 e, broadcast
+//    reads), packed fp32x2 FMA.  Online softmax per head with a warp max.
+//  * PV: lane owns d_v / 32 output channels for every head of the unit; the
+//    per-token probabilities are broadcast from shared memory.
+//  * When a warp's range leaves a unit it writes its partial (max, sum, o) for
+//    that unit; a merge kernel combines the partials of each head by
+//    log-sum-exp and writes out / lse.
+#include <algorithm>
+
+#include "tls_device.cuh"
+#include "tls_internal.h"
+
+namespace tls {
+namespace {
+
+constexpr int kTT = 32;  // tokens per tile
+
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+template <typename E, int D, int DV, int HG, bool VPREFIX, int W, int NS>
+struct AttnLayout {
+  static constexpr int kElt = E::kBytes;
+  static constexpr int RB = D * kElt;                     // K row bytes
+  static constexpr int KCH = RB / 16;                     // 16-byte chunks per K row
+  static constexpr int VB = VPREFIX ? 0 : DV * kElt;      // V row bytes (0: V inside K row)
+  static constexpr int VCH = VB / 16;
+  static constexpr int CPL = DV / 32;                     // output channels per lane
+  static constexpr int kStageBytes = kTT * (RB + VB);
+  static constexpr int kWarpBytes = NS * kStageBytes + HG * D * 4 + kTT * HG * 4 + NS * kTT * 8;
+  static constexpr int kSmem = W * kWarpBytes;
+  static_assert(KCH % 8 == 0, "row must be a multiple of 128 bytes for the swizzle");
+  static_assert(DV % 32 == 0, "d_v must be a multiple of 32");
+};
+
+template <typename E, int D, int DV, int HG, bool VPREFIX, bool PAGED, int W, int NS>
+__global__ void __launch_bounds__(W * 32, 1) attn_split_kernel(AttnArgs a, AttnPlan p) {
+  using L = AttnLayout<E, D, DV, HG, VPREFIX, W, NS>;
+  using S = typename E::storage;
+  constexpr int EPC = E::kEPC;
+  constexpr int CPL = L::CPL;
+  extern __shared__ __align__(128) unsigned char smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned char *wbase = smem + warp * L::kWarpBytes;
+  unsigned char *stage_base = wbase;                                        // NS stages
+  float *Qs = reinterpret_cast<float *>(wbase + NS * L::kStageBytes);       // [HG][D]
+  float *Ps = Qs + HG * D;                                                  // [kTT][HG]
+  long long *Off = reinterpret_cast<long long *>(Ps + kTT * HG);            // [NS][kTT]
+
+  const int gw = blockIdx.x * W + warp;
+  const int t_begin = gw * p.tiles_per_warp;
+  const int t_end = min(t_begin + p.tiles_per_warp, p.total_tiles);
+  if (t_begin >= t_end) return;
+
+  const S *Kb = static_cast<const S *>(a.K);
+  const S *Vb = VPREFIX ? Kb : (PAGED ? Kb : static_cast<const S *>(a.V));
+  const int Gt = a.n_q_heads / a.n_kv_heads;
+
+  // Gather the rows of tile t into stage st (always commits one group).
+  auto issue = [&](int t, int st) {
+    if (t < t_end) {
+      const int unit = t / p.tiles_per_group, tile = t % p.tiles_per_group;
+      const int group = unit / p.n_head_chunks;
+      const int j = tile * kTT + lane;
+      long long off = -1;
+      if (j < a.k_t) {
+        const int tok = a.token_idx[static_cast<size_t>(group) * a.k_t + j];
+        if (tok >= 0 && tok < a.max_ctx) {
+          if constexpr (PAGED) {
+            const int slot = a.slot_of_block[static_cast<size_t>(group) * a.n_blocks_max + tok / a.block_size];
+            if (slot >= 0 && slot < a.n_slots)
+              off = ((static_cast<long long>(group) * a.n_slots + slot) * 2 * a.block_size + tok % a.block_size) * D;
+          } else {
+            off = (static_cast<long long>(group) * a.max_ctx + tok) * D;
+          }
+        }
+      }
+      Off[st * kTT + lane] = off;
+      __syncwarp();
+      unsigned char *Ks = stage_base + st * L::kStageBytes;
+#pragma unroll 4
+      for (int idx = lane; idx < kTT * L::KCH; idx += 32) {
+        const int row = idx / L::KCH, c = idx % L::KCH;
+        const long long o = Off[st * kTT + row];
+        const S *src = Kb + (o >= 0 ? o : 0) + c * EPC;
+        cp_async16(Ks + row * L::RB + ((c ^ (row & 7)) * 16), src, o >= 0);
+      }
+      if constexpr (!VPREFIX) {
+        unsigned char *Vs = Ks + kTT * L::RB;
+#pragma unroll 4
+        for (int idx = lane; idx < kTT * L::VCH; idx += 32) {
+          const int row = idx / L::VCH, c = idx % L::VCH;
+          const long long o = Off[st * kTT + row];
+          const long long vo = PAGED ? o + static_cast<long long>(a.block_size) * D : o;
+          const S *src = Vb + (o >= 0 ? vo : 0) + c * EPC;
+          cp_async16(Vs + row * L::VB + c * 16, src, o >= 0);
+        }
+      }
+    }
+    cp_async_commit();
+  };
+
+  float m[HG], l[HG], acc[HG][CPL];
+  int cur_unit = -1;
+
+  auto reset = [&]() {
+#pragma unroll
+    for (int h = 0; h < HG; ++h) {
+      m[h] = -INFINITY;
+      l[h] = 0.f;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) acc[h][c] = 0.f;
+    }
+  };
+
+  auto flush = [&](int unit) {
+    const int first = (unit * p.tiles_per_group) / p.tiles_per_warp;
+    const int piece = gw - first;
+    float *ml = a.part + (static_cast<size_t>(unit) * p.max_pieces + piece) * HG * 2;
+    float *po = a.part + static_cast<size_t>(a.batch) * a.n_kv_heads * p.n_head_chunks * p.max_pieces * HG * 2 +
+                (static_cast<size_t>(unit) * p.max_pieces + piece) * HG * DV;
+#pragma unroll
+    for (int h = 0; h < HG; ++h) {
+      const float lt = warp_sum(l[h]);
+      if (lane == 0) { ml[h * 2] = m[h]; ml[h * 2 + 1] = lt; }
+      float *dst = po + h * DV + lane * CPL;
+#pragma unroll
+      for (int c = 0; c < CPL; c += 2) *reinterpret_cast<float2 *>(dst + c) = make_float2(acc[h][c], acc[h][c + 1]);
+    }
+  };
+
+  auto load_q = [&](int unit) {
+    const int group = unit / p.n_head_chunks, hc = unit % p.n_head_chunks;
+    const int b = group / a.n_kv_heads, g = group % a.n_kv_heads;
+    const size_t q0 = (static_cast<size_t>(b) * a.n_q_heads + g * Gt + hc * HG) * D;
+    for (int i = lane; i < HG * D; i += 32) Qs[i] = load_elem<E>(a.q, q0 + i) * a.scale_log2;
+    __syncwarp();
+  };
+
+#pragma unroll
+  for (int s = 0; s < NS - 1; ++s) issue(t_begin + s, s);
+
+  for (int t = t_begin; t < t_end; ++t) {
+    const int st = (t - t_begin) % NS;
+    issue(t + NS - 1, (t + NS - 1 - t_begin) % NS);
+    cp_async_wait<NS - 1>();
+    __syncwarp();
+    const int unit = t / p.tiles_per_group;
+    if (unit != cur_unit) {
+      if (cur_unit >= 0) flush(cur_unit);
+      reset();
+      load_q(unit);
+      cur_unit = unit;
+    }
+    const unsigned char *Ks = stage_base + st * L::kStageBytes;
+    const bool valid = Off[st * kTT + lane] >= 0;
+
+    // ---- scores: lane = token row
+    float2 s2[HG];
+#pragma unroll
+    for (int h = 0; h < HG; ++h) s2[h] = make_float2(0.f, 0.f);
+    const unsigned char *krow = Ks + lane * L::RB;
+#pragma unroll 8
+    for (int j = 0; j < L::KCH; ++j) {
+      const uint4 kc = *reinterpret_cast<const uint4 *>(krow + ((j ^ (lane & 7)) * 16));
+      float kf[EPC];
+      chunk_to_f32<E>(kc, kf);
+#pragma unroll
+      for (int h = 0; h < HG; ++h) {
+        const float4 *qp = reinterpret_cast<const float4 *>(Qs + h * D + j * EPC);
+#pragma unroll
+        for (int e = 0; e < EPC / 4; ++e) {
+          const float4 qv = qp[e];
+          ffma2(s2[h], make_float2(kf[4 * e], kf[4 * e + 1]), make_float2(qv.x, qv.y));
+          ffma2(s2[h], make_float2(kf[4 * e + 2], kf[4 * e + 3]), make_float2(qv.z, qv.w));
+        }
+      }
+    }
+    // ---- online softmax (log2 domain)
+#pragma unroll
+    for (int h = 0; h < HG; ++h) {
+      const float sc = valid ? (s2[h].x + s2[h].y) : -INFINITY;
+      const float mn = fmaxf(m[h], warp_max(sc));
+      float alpha = 1.f, pr = 0.f;
+      if (mn != -INFINITY) {
+        alpha = ex2(m[h] - mn);
+        pr = ex2(sc - mn);
+      }
+      l[h] = l[h] * alpha + pr;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) acc[h][c] *= alpha;
+      m[h] = mn;
+      Ps[lane * HG + h] = pr;
+    }
+    __syncwarp();
+    // ---- o += p v: lane owns channels [lane*CPL, lane*CPL + CPL)
+    const unsigned char *Vs = VPREFIX ? Ks : Ks + kTT * L::RB;
+#pragma unroll 4
+    for (int r = 0; r < kTT; ++r) {
+      float pv[HG];
+#pragma unroll
+      for (int h = 0; h < HG; ++h) pv[h] = Ps[r * HG + h];
+      float vf[CPL];
+      if constexpr (VPREFIX) {
+        // channels lane*CPL.. live in K-row chunks (swizzled)
+#pragma unroll
+        for (int q = 0; q < CPL / EPC; ++q) {
+          const int c = lane * (CPL / EPC) + q;
+          const uint4 vc = *reinterpret_cast<const uint4 *>(Vs + r * L::RB + ((c ^ (r & 7)) * 16));
+          chunk_to_f32<E>(vc, vf + q * EPC);
+        }
+      } else {
+        const unsigned char *vr = Vs + r * L::VB + lane * CPL * L::kElt;
+        if constexpr (CPL * L::kElt == 16) {
+          chunk_to_f32<E>(*reinterpret_cast<const uint4 *>(vr), vf);
+        } else if constexpr (CPL * L::kElt == 8) {
+          const uint2 w = *reinterpret_cast<const uint2 *>(vr);
+          if constexpr (sizeof(S) == 2) {
+            vf[0] = bf16_lo(w.x); vf[1] = bf16_hi(w.x); vf[2] = bf16_lo(w.y); vf[3] = bf16_hi(w.y);
+          } else {
+            vf[0] = __uint_as_float(w.x); vf[1] = __uint_as_float(w.y);
+          }
+        } else {
+          static_assert(CPL * L::kElt == 4, "unsupported V slice");
+          const uint32_t w = *reinterpret_cast<const uint32_t *>(vr);
+          vf[0] = bf16_lo(w); vf[1] = bf16_hi(w);
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < HG; ++h) {
+#pragma unroll
+        for (int c = 0; c < CPL; c += 2) {
+          float2 o2 = make_float2(acc[h][c], acc[h][c + 1]);
+          ffma2(o2, make_float2(vf[c], vf[c + 1]), make_float2(pv[h], pv[h]));
+          acc[h][c] = o2.x;
+          acc[h][c + 1] = o2.y;
+        }
+      }
+    }
+    __syncwarp();
+  }
+  if (cur_unit >= 0) flush(cur_unit);
+  cp_async_wait<0>();
+}
+
+template <int DV, int HG>
+__global__ void __launch_bounds__(128) attn_merge_kernel(AttnArgs a, AttnPlan p) {
+  constexpr int CPL = DV / 32;
+  const int lane = threadIdx.x & 31;
+  const int w = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int n_units = a.batch * a.n_kv_heads * p.n_head_chunks;
+  if (w >= n_units * HG) return;
+  const int unit = w / HG, hh = w % HG;
+  const int group = unit / p.n_head_chunks, hc = unit % p.n_head_chunks;
+  const int b = group / a.n_kv_heads, g = group % a.n_kv_heads;
+  const int Gt = a.n_q_heads / a.n_kv_heads;
+  const int head = g * Gt + hc * HG + hh;
+  const int first = (unit * p.tiles_per_group) / p.tiles_per_warp;
+  const int last = ((unit + 1) * p.tiles_per_group - 1) / p.tiles_per_warp;
+  const float *ml = a.part + static_cast<size_t>(unit) * p.max_pieces * HG * 2;
+  const float *po = a.part + static_cast<size_t>(n_units) * p.max_pieces * HG * 2 +
+                    static_cast<size_t>(unit) * p.max_pieces * HG * DV;
+  float M = -INFINITY;
+  for (int q = 0; q <= last - first; ++q) M = fmaxf(M, ml[(q * HG + hh) * 2]);
+  float o[CPL];
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) o[c] = 0.f;
+  float Lsum = 0.f;
+  if (M != -INFINITY) {
+    for (int q = 0; q <= last - first; ++q) {
+      const float wq = ex2(ml[(q * HG + hh) * 2] - M);
+      Lsum += wq * ml[(q * HG + hh) * 2 + 1];
+      const float *src = po + (static_cast<size_t>(q) * HG + hh) * DV;
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) o[c] += wq * src[c * 32 + lane];
+    }
+  }
+  const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+  const size_t ob = (static_cast<size_t>(b) * a.n_q_heads + head) * DV;
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) {
+    const float v = o[c] * inv;
+    if (a.out_dtype == 1) static_cast<uint16_t *>(a.out)[ob + c * 32 + lane] = f32_to_bf16_rne(v);
+    else static_cast<float *>(a.out)[ob + c * 32 + lane] = v;
+  }
+  if (a.lse && lane == 0)
+    a.lse[static_cast<size_t>(b) * a.n_q_heads + head] =
+        (M == -INFINITY || Lsum <= 0.f) ? -INFINITY : (M + log2f(Lsum)) * 0.69314718055994531f;
+}
+
+template <typename E, int D, int DV, int HG, bool VPREFIX, bool PAGED, int W, int NS>
+cudaError_t run_attention(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) {
+  using L = AttnLayout<E, D, DV, HG, VPREFIX, W, NS>;
+  auto kern = attn_split_kernel<E, D, DV, HG, VPREFIX, PAGED, W, NS>;
+  static bool configured[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !configured[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kSmem);
+    if (e != cudaSuccess) return e;
+    configured[dev] = true;
+  }
+  kern<<<p.grid, W * 32, L::kSmem, st>>>(a, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int n_warps = a.batch * a.n_kv_heads * p.n_head_chunks * HG;
+  attn_merge_kernel<DV, HG><<<(n_warps + 3) / 4, 128, 0, st>>>(a, p);
+  return cudaGetLastError();
+}
+
+// Kernel-set selection.  Returns false for shapes outside the compiled set.
+struct Variant {
+  int warps, stages, head_chunk;
+};
+
+bool pick_variant(const AttnArgs &a, Variant *v) {
+  const int G = a.n_q_heads / a.n_kv_heads;
+  if (a.v_is_k_prefix) {
+    if (a.dtype != 1 || a.d_qk != 576 || a.d_v != 512 || a.paged) return false;
+    if (G % 4 != 0 || G > 128) return false;
+    *v = {2, 2, 4};
+    return true;
+  }
+  if (a.d_qk != a.d_v || (a.d_qk != 64 && a.d_qk != 128)) return false;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return false;
+  const int rb = a.d_qk * (a.dtype == 1 ? 2 : 4);
+  if (rb == 128) *v = {8, 3, G};
+  else if (rb == 256) *v = {4, 3, G};
+  else *v = {3, 2, G};
+  return true;
+}
+
+template <typename E, int D, bool PAGED>
+cudaError_t dispatch_gqa(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) {
+  constexpr int RB = D * E::kBytes;
+  constexpr int W = RB == 128 ? 8 : (RB == 256 ? 4 : 3);
+  constexpr int NS = RB == 512 ? 2 : 3;
+  switch (p.head_chunk) {
+    case 1: return run_attention<E, D, D, 1, false, PAGED, W, NS>(a, p, st);
+    case 2: return run_attention<E, D, D, 2, false, PAGED, W, NS>(a, p, st);
+    case 4: return run_attention<E, D, D, 4, false, PAGED, W, NS>(a, p, st);
+    case 8: return run_attention<E, D, D, 8, false, PAGED, W, NS>(a, p, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+bool attn_plan(const AttnArgs &a, AttnPlan *p) {
+  Variant v;
+  if (!pick_variant(a, &v)) return false;
+  const int G = a.n_q_heads / a.n_kv_heads;
+  p->warps_per_cta = v.warps;
+  p->tokens_per_tile = kTT;
+  p->head_chunk = v.head_chunk;
+  p->n_head_chunks = G / v.head_chunk;
+  const long long units = static_cast<long long>(a.batch) * a.n_kv_heads * p->n_head_chunks;
+  p->tiles_per_group = (a.k_t + kTT - 1) / kTT;
+  const long long total = units * p->tiles_per_group;
+  if (total <= 0 || total > (1LL << 30)) return false;
+  p->total_tiles = static_cast<int>(total);
+  const int sms = a.num_sms > 0 ? a.num_sms : 148;
+  p->grid = static_cast<int>(std::min<long long>(sms, (total + v.warps - 1) / v.warps));
+  const long long nw = static_cast<long long>(p->grid) * v.warps;
+  p->tiles_per_warp = static_cast<int>((total + nw - 1) / nw);
+  p->max_pieces = (p->tiles_per_group + p->tiles_per_warp - 1) / p->tiles_per_warp + 1;
+  p->part_floats = static_cast<size_t>(units) * p->max_pieces * p->head_chunk * (2 + a.d_v);
+  return true;
+}
+
+cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) {
+  if (a.v_is_k_prefix) return run_attention<BF16, 576, 512, 4, true, false, 2, 2>(a, p, st);
+  if (a.dtype == 1) {
+    if (a.d_qk == 128) return a.paged ? dispatch_gqa<BF16, 128, true>(a, p, st) : dispatch_gqa<BF16, 128, false>(a, p, st);
+    return a.paged ? dispatch_gqa<BF16, 64, true>(a, p, st) : dispatch_gqa<BF16, 64, false>(a, p, st);
+  }
+  if (a.d_qk == 128) return a.paged ? dispatch_gqa<F32, 128, true>(a, p, st) : dispatch_gqa<F32, 128, false>(a, p, st);
+  return a.paged ? dispatch_gqa<F32, 64, true>(a, p, st) : dispatch_gqa<F32, 64, false>(a, p, st);
+}
+
+}  // namespace tls

@@ -1,0 +1,86 @@
+// tls_internal.h -- host-side launchers of the libtls kernels (internal, not ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace tls {
+
+constexpr int kMaxSelectKeys = 16384;  // keys held in shared memory by one selection CTA
+
+struct MetaArgs {
+  const void *K;
+  const int32_t *seq_lens;
+  const int32_t *label_idx;
+  void *meta;
+  void *slab;
+  int batch, n_kv_heads, d, block_size, n_blocks_max, max_ctx, n_label, dtype;
+};
+cudaError_t launch_build_meta(const MetaArgs &a, cudaStream_t st);
+cudaError_t launch_build_slab(const MetaArgs &a, cudaStream_t st);
+
+struct BlockScoreArgs {
+  const void *q;
+  const void *meta;
+  const int32_t *seq_lens;
+  float *scores;      // [B*H_kv][n_blocks_max]
+  int32_t *block_idx; // [B*H_kv][k_b]
+  int batch, n_q_heads, n_kv_heads, d, block_size, n_blocks_max, max_ctx, k_b, dtype;
+  int num_sms;
+};
+cudaError_t launch_block_score(const BlockScoreArgs &a, cudaStream_t st);
+cudaError_t launch_block_topk(const BlockScoreArgs &a, cudaStream_t st);
+
+struct TokenArgs {
+  const void *q;
+  const void *slab;
+  const int32_t *label_idx;
+  const int32_t *block_idx;
+  const int32_t *seq_lens;
+  int32_t *token_idx;
+  float *token_score;  // nullable
+  int batch, n_q_heads, n_kv_heads, d, block_size, n_blocks_max, max_ctx, n_label, k_b, k_t, dtype;
+};
+cudaError_t launch_token_topk(const TokenArgs &a, cudaStream_t st);
+
+struct AttnArgs {
+  const void *q;
+  const void *K;
+  const void *V;
+  const int32_t *token_idx;
+  const int32_t *slot_of_block;  // paged only
+  int n_slots;                   // paged only
+  void *out;
+  float *lse;
+  float *part;  // workspace partials
+  int batch, n_q_heads, n_kv_heads, d_qk, d_v, v_is_k_prefix, block_size, n_blocks_max, max_ctx, k_t;
+  int dtype, out_dtype, paged;
+  float scale_log2;  // softmax_scale * log2(e)
+  int num_sms;
+};
+// Partial-result layout chosen for a shape on a device; shared by the
+// workspace query and the launch so both agree.
+struct AttnPlan {
+  int warps_per_cta, tokens_per_tile, head_chunk, n_head_chunks;
+  int tiles_per_group, total_tiles, grid, tiles_per_warp, max_pieces;
+  size_t part_floats;  // floats of workspace for partials
+};
+bool attn_plan(const AttnArgs &a, AttnPlan *p);
+cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &p, cudaStream_t st);
+
+struct OffloadArgs {
+  const void *host_kv;  // device-visible pointer of the pinned host KV
+  void *cache;
+  int32_t *slot_of_block;
+  int32_t *block_of_slot;
+  const int32_t *prev_block_idx;
+  const int32_t *next_block_idx;
+  int32_t *n_new;
+  int32_t *jobs;
+  int batch, n_kv_heads, d, block_size, n_blocks_max, k_b, n_slots, dtype;
+};
+cudaError_t launch_offload_reset(const OffloadArgs &a, cudaStream_t st);
+cudaError_t launch_prefetch_diff(const OffloadArgs &a, cudaStream_t st);
+
+}  // namespace tls

@@ -1,0 +1,90 @@
+// tls_meta.cu -- set-up kernels: per-block channel max/min summary and the
+// label-channel slab (AsyncTLS block summary "Max/Min der Keys", gist.science
+// (de) section 2.A "Stufe 1"; label channels, (es) section 2.A.2).
+//
+// build_meta: one thread owns one 16-byte chunk of channels of one block and
+// walks the block's valid tokens; a warp reads 512 contiguous bytes per token
+// step.  The max / min of stored values is itself a stored value, so the
+// summary is exact in the storage type.
+// build_slab: one thread per (token, label channel); coalesced slab writes.
+#include "tls_device.cuh"
+#include "tls_internal.h"
+
+namespace tls {
+namespace {
+
+template <typename E>
+__global__ void __launch_bounds__(256) build_meta_kernel(MetaArgs a) {
+  constexpr int EPC = E::kEPC;
+  const int chunks = a.d / EPC;  // 16-byte chunks per key row
+  const int group = blockIdx.y;  // b * H_kv + g
+  const int b = group / a.n_kv_heads;
+  const int seq = min(max(a.seq_lens[b], 0), a.max_ctx);
+  const long long item = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int blk = static_cast<int>(item / chunks), c = static_cast<int>(item % chunks);
+  if (blk >= a.n_blocks_max) return;
+  const int t0 = blk * a.block_size, t1 = min(t0 + a.block_size, seq);
+  if (t0 >= t1) return;  // no valid token: left untouched
+  using S = typename E::storage;
+  const S *K = static_cast<const S *>(a.K) + (static_cast<size_t>(group) * a.max_ctx) * a.d + c * EPC;
+  float hi[EPC], lo[EPC];
+#pragma unroll
+  for (int e = 0; e < EPC; ++e) { hi[e] = -INFINITY; lo[e] = INFINITY; }
+  for (int t = t0; t < t1; ++t) {
+    uint4 v = ld_stream16(K + static_cast<size_t>(t) * a.d);
+    float f[EPC];
+    chunk_to_f32<E>(v, f);
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) { hi[e] = fmaxf(hi[e], f[e]); lo[e] = fminf(lo[e], f[e]); }
+  }
+  S *m = static_cast<S *>(a.meta) + ((static_cast<size_t>(group) * a.n_blocks_max + blk) * 2) * a.d + c * EPC;
+  S ho[EPC], lw[EPC];
+#pragma unroll
+  for (int e = 0; e < EPC; ++e) {
+    if constexpr (sizeof(S) == 2) {
+      ho[e] = static_cast<S>(__float_as_uint(hi[e]) >> 16);  // exact: the value came from a bf16
+      lw[e] = static_cast<S>(__float_as_uint(lo[e]) >> 16);
+    } else {
+      ho[e] = hi[e];
+      lw[e] = lo[e];
+    }
+  }
+  *reinterpret_cast<uint4 *>(m) = *reinterpret_cast<const uint4 *>(ho);
+  *reinterpret_cast<uint4 *>(m + a.d) = *reinterpret_cast<const uint4 *>(lw);
+}
+
+template <typename E>
+__global__ void __launch_bounds__(256) build_slab_kernel(MetaArgs a) {
+  using S = typename E::storage;
+  const int group = blockIdx.y;
+  const int b = group / a.n_kv_heads;
+  const int seq = min(max(a.seq_lens[b], 0), a.max_ctx);
+  const long long item = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int t = static_cast<int>(item / a.n_label), c = static_cast<int>(item % a.n_label);
+  if (t >= seq) return;
+  const int ch = a.label_idx[c];
+  const S *K = static_cast<const S *>(a.K) + (static_cast<size_t>(group) * a.max_ctx + t) * a.d;
+  S v = (ch >= 0 && ch < a.d) ? K[ch] : S(0);
+  static_cast<S *>(a.slab)[(static_cast<size_t>(group) * a.max_ctx + t) * a.n_label + c] = v;
+}
+
+}  // namespace
+
+cudaError_t launch_build_meta(const MetaArgs &a, cudaStream_t st) {
+  const int epc = a.dtype == 1 ? BF16::kEPC : F32::kEPC;
+  const long long items = static_cast<long long>(a.n_blocks_max) * (a.d / epc);
+  dim3 grid(static_cast<unsigned>((items + 255) / 256), a.batch * a.n_kv_heads);
+  if (a.dtype == 1) build_meta_kernel<BF16><<<grid, 256, 0, st>>>(a);
+  else build_meta_kernel<F32><<<grid, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_build_slab(const MetaArgs &a, cudaStream_t st) {
+  const long long items = static_cast<long long>(a.max_ctx) * a.n_label;
+  dim3 grid(static_cast<unsigned>((items + 255) / 256), a.batch * a.n_kv_heads);
+  if (a.dtype == 1) build_slab_kernel<BF16><<<grid, 256, 0, st>>>(a);
+  else build_slab_kernel<F32><<<grid, 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace tls

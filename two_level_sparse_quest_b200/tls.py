@@ -1,0 +1,192 @@
+"""ctypes binding of libtls.so (include/tls.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls, takes torch
+tensors (or raw integer pointers) and passes their device pointers, sizes and
+the CUDA stream through unchanged.  No step of the decode path runs in Python;
+a missing library raises ImportError at import time, and a failing call raises
+TlsError with the library's message.  There is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtls.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built; run `python -m two_level_sparse_quest_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+TLS_OK, TLS_ERR_INVALID_ARG, TLS_ERR_UNSUPPORTED, TLS_ERR_WORKSPACE, TLS_ERR_CUDA, TLS_ERR_TIMEOUT = range(6)
+TLS_F32, TLS_BF16 = 0, 1
+STATUS_NAMES = {0: "TLS_OK", 1: "TLS_ERR_INVALID_ARG", 2: "TLS_ERR_UNSUPPORTED", 3: "TLS_ERR_WORKSPACE",
+                4: "TLS_ERR_CUDA", 5: "TLS_ERR_TIMEOUT"}
+
+EXPORTED = ("tls_version", "tls_last_error", "tls_workspace_size", "tls_build_block_meta", "tls_block_score_topk",
+            "tls_token_score_topk", "tls_sparse_attn_decode", "tls_sparse_attn_decode_paged", "tls_offload_reset",
+            "tls_prefetch_diff", "tls_wait_event")
+
+
+class TlsShape(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "batch", "n_q_heads", "n_kv_heads", "d_qk", "d_v", "v_is_k_prefix", "block_size", "n_label",
+        "k_b", "k_t", "max_ctx", "kv_dtype", "out_dtype")] + [("softmax_scale", ctypes.c_float)]
+
+    def __repr__(self):
+        return "TlsShape(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+class TlsError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+_P = ctypes.c_void_p
+_S = ctypes.POINTER(TlsShape)
+_i32 = ctypes.c_int32
+_sz = ctypes.c_size_t
+_sigs = {
+    "tls_version": ([], ctypes.c_char_p),
+    "tls_last_error": ([], ctypes.c_char_p),
+    "tls_workspace_size": ([_S], _sz),
+    "tls_build_block_meta": ([_S, _P, _P, _P, _P, _P, _P], ctypes.c_int),
+    "tls_block_score_topk": ([_S, _P, _P, _P, _P, _P, _P, _sz, _P], ctypes.c_int),
+    "tls_token_score_topk": ([_S, _P, _P, _P, _P, _P, _P, _P, _P, _sz, _P], ctypes.c_int),
+    "tls_sparse_attn_decode": ([_S, _P, _P, _P, _P, _P, _P, _P, _sz, _P], ctypes.c_int),
+    "tls_sparse_attn_decode_paged": ([_S, _P, _P, _P, _i32, _P, _P, _P, _P, _sz, _P], ctypes.c_int),
+    "tls_offload_reset": ([_S, _i32, _P, _P, _P], ctypes.c_int),
+    "tls_prefetch_diff": ([_S, _i32, _P, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
+    "tls_wait_event": ([_P, _i32], ctypes.c_int),
+}
+for _name, (_args, _ret) in _sigs.items():
+    _f = getattr(_lib, _name)
+    _f.argtypes = _args
+    _f.restype = _ret
+
+
+def make_shape(batch, n_q_heads, n_kv_heads, d_qk, d_v, block_size, n_label, k_b, k_t, max_ctx, kv_dtype,
+               out_dtype=TLS_F32, v_is_k_prefix=False, softmax_scale: Optional[float] = None) -> TlsShape:
+    s = TlsShape()
+    s.batch, s.n_q_heads, s.n_kv_heads = batch, n_q_heads, n_kv_heads
+    s.d_qk, s.d_v, s.v_is_k_prefix = d_qk, d_v, int(bool(v_is_k_prefix))
+    s.block_size, s.n_label, s.k_b, s.k_t, s.max_ctx = block_size, n_label, k_b, k_t, max_ctx
+    s.kv_dtype, s.out_dtype = kv_dtype, out_dtype
+    s.softmax_scale = (1.0 / math.sqrt(d_qk)) if softmax_scale is None else softmax_scale
+    return s
+
+
+def shape_from_workload(w, out_dtype=TLS_F32, **over) -> TlsShape:
+    kw = dict(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, d_qk=w.d_qk, d_v=w.d_v,
+              block_size=w.block_size, n_label=w.n_label, k_b=w.k_b, k_t=w.k_t, max_ctx=w.ctx, kv_dtype=w.dtype,
+              out_dtype=out_dtype, v_is_k_prefix=w.v_is_k_prefix)
+    kw.update(over)
+    return make_shape(**kw)
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if isinstance(x, torch.Tensor):
+        if not x.is_contiguous():
+            raise ValueError("tensor must be contiguous")
+        return x.data_ptr()
+    raise TypeError(f"expected a tensor, an int pointer or None, got {type(x)}")
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _ws(ws):
+    if ws is None:
+        return None, 0
+    if isinstance(ws, tuple):
+        return ws
+    return ws.data_ptr(), ws.numel() * ws.element_size()
+
+
+def _check(st: int, name: str):
+    if st != TLS_OK:
+        raise TlsError(st, f"{name}: {tls_last_error()}")
+
+
+def tls_version() -> str:
+    return _lib.tls_version().decode()
+
+
+def tls_last_error() -> str:
+    return _lib.tls_last_error().decode()
+
+
+def tls_workspace_size(shape: TlsShape) -> int:
+    n = _lib.tls_workspace_size(ctypes.byref(shape))
+    if n == 0:
+        raise TlsError(TLS_ERR_UNSUPPORTED, f"tls_workspace_size: {tls_last_error()}")
+    return n
+
+
+def tls_build_block_meta(shape, K, seq_lens, label_idx, meta_out, slab_out=None, stream=None):
+    _check(_lib.tls_build_block_meta(ctypes.byref(shape), _ptr(K), _ptr(seq_lens), _ptr(label_idx), _ptr(meta_out),
+                                     _ptr(slab_out), _stream(stream)), "tls_build_block_meta")
+
+
+def tls_block_score_topk(shape, q, meta, seq_lens, block_idx_out, block_score_out=None, ws=None, stream=None):
+    wp, wb = _ws(ws)
+    _check(_lib.tls_block_score_topk(ctypes.byref(shape), _ptr(q), _ptr(meta), _ptr(seq_lens), _ptr(block_idx_out),
+                                     _ptr(block_score_out), wp, wb, _stream(stream)), "tls_block_score_topk")
+
+
+def tls_token_score_topk(shape, q, slab, label_idx, block_idx, seq_lens, token_idx_out, token_score_out=None,
+                         ws=None, stream=None):
+    wp, wb = _ws(ws)
+    _check(_lib.tls_token_score_topk(ctypes.byref(shape), _ptr(q), _ptr(slab), _ptr(label_idx), _ptr(block_idx),
+                                     _ptr(seq_lens), _ptr(token_idx_out), _ptr(token_score_out), wp, wb,
+                                     _stream(stream)), "tls_token_score_topk")
+
+
+def tls_sparse_attn_decode(shape, q, K, V, token_idx, out, lse_out=None, ws=None, stream=None):
+    wp, wb = _ws(ws)
+    _check(_lib.tls_sparse_attn_decode(ctypes.byref(shape), _ptr(q), _ptr(K), _ptr(V), _ptr(token_idx), _ptr(out),
+                                       _ptr(lse_out), wp, wb, _stream(stream)), "tls_sparse_attn_decode")
+
+
+def tls_sparse_attn_decode_paged(shape, q, cache, slot_of_block, n_slots, token_idx, out, lse_out=None, ws=None,
+                                 stream=None):
+    wp, wb = _ws(ws)
+    _check(_lib.tls_sparse_attn_decode_paged(ctypes.byref(shape), _ptr(q), _ptr(cache), _ptr(slot_of_block),
+                                             int(n_slots), _ptr(token_idx), _ptr(out), _ptr(lse_out), wp, wb,
+                                             _stream(stream)), "tls_sparse_attn_decode_paged")
+
+
+def tls_offload_reset(shape, n_slots, slot_of_block, block_of_slot, stream=None):
+    _check(_lib.tls_offload_reset(ctypes.byref(shape), int(n_slots), _ptr(slot_of_block), _ptr(block_of_slot),
+                                  _stream(stream)), "tls_offload_reset")
+
+
+def tls_prefetch_diff(shape, n_slots, host_kv, cache, slot_of_block, block_of_slot, prev_block_idx, next_block_idx,
+                      n_new_out, jobs_ws, stream=None):
+    _check(_lib.tls_prefetch_diff(ctypes.byref(shape), int(n_slots), _ptr(host_kv), _ptr(cache), _ptr(slot_of_block),
+                                  _ptr(block_of_slot), _ptr(prev_block_idx), _ptr(next_block_idx), _ptr(n_new_out),
+                                  _ptr(jobs_ws), _stream(stream)), "tls_prefetch_diff")
+
+
+def tls_wait_event(event, timeout_ms: int) -> int:
+    """Returns the status (TLS_OK or TLS_ERR_TIMEOUT); raises on other errors."""
+    handle = event if isinstance(event, int) else event.cuda_event
+    st = _lib.tls_wait_event(handle, int(timeout_ms))
+    if st not in (TLS_OK, TLS_ERR_TIMEOUT):
+        _check(st, "tls_wait_event")
+    return st
