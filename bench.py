@@ -30,7 +30,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "sparse-attn decode steps/sec (all heads) at 96k ctx; achieved HBM GB/s vs peak"
-N_LAYERS = 4
+N_LAYERS_DEFAULT = 4
 SMI_FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -151,6 +151,24 @@ class ClockSampler:
                 "samples": len(sm), "power_w_max": max(power) if power else None}
 
 
+# ----------------------------------------------------------------------------- ranks
+def rank_workload(base, rank: int):
+    """Weak scaling: rank r decodes its own independent sequences (seed offset)."""
+    return base.with_(seed=base.seed + 7919 * rank)
+
+
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank timing over all ranks (the job's time)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ----------------------------------------------------------------------------- GPU arm
 class Layer:
     """One layer's resident state: KV cache, block summary, label slab, query."""
@@ -181,9 +199,10 @@ def gpu_arm(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     base = W.WORKLOADS[args.workload]
-    w = base.with_(seed=base.seed + 7919 * rank)  # each rank: its own sequences
+    w = rank_workload(base, rank)
     shape = T.shape_from_workload(w)
     inp = W.make_decode_inputs(w)
+    N_LAYERS = args.layers
     qs = W.make_query_stream(w.with_(ar_rho=0.5), steps=N_LAYERS)
 
     def up(a):
@@ -226,8 +245,8 @@ def gpu_arm(args, rank, world, local_rank):
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local_rank)).split(",")[0])
-                           if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit() else local_rank)
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+    sampler = ClockSampler(int(vis[local_rank]) if local_rank < len(vis) and vis[local_rank].isdigit() else local_rank)
     if rank == 0:
         sampler.start()
     if world > 1:
@@ -246,10 +265,7 @@ def gpu_arm(args, rank, world, local_rank):
     ms = t_start.elapsed_time(t_end)
     st = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])] for e in evs])
     stage_ms = st.mean(axis=0)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, dev)
 
     # ---- end to end through the C ABI with host buffers: H2D q, step, D2H out + lse
     n_e2e = min(args.steps, 500)
@@ -279,10 +295,7 @@ def gpu_arm(args, rank, world, local_rank):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev)
     h2d = layers[0].q.numel() * layers[0].q.element_size()
     d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
 
@@ -395,6 +408,8 @@ def main():
     ap.add_argument("--workload", default="gqa96k_b8_bf16")
     ap.add_argument("--impl", default="tls", choices=["tls", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=N_LAYERS_DEFAULT,
+                    help="layer copies rotated through (4 keeps the per-rotation working set above L2)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
