@@ -211,6 +211,25 @@ TLS_API tls_status tls_prefetch_diff(const tls_shape *s, int32_t n_slots, const 
                              int32_t *slot_of_block, int32_t *block_of_slot, const int32_t *prev_block_idx,
                              const int32_t *next_block_idx, int32_t *n_new_out, int32_t *jobs_ws, void *stream);
 
+/* Stages 1+2 for callers that cannot allocate device memory (no counterpart in
+ * the paper: an addition of this library).  Computes exactly what
+ * tls_block_score_topk computes with block_score_out = NULL, but keeps the fp32
+ * block scores in a fixed 4 MiB array inside the library's own device memory
+ * instead of a caller workspace, so a caller that may not call cudaMalloc and
+ * has no spare device buffer (e.g. code running inside another runtime's
+ * launch hook) needs only the inputs and block_idx_out.
+ *   Limit: batch * n_kv_heads * ceil(max_ctx / block_size) <= 1048576 block
+ *   scores; larger shapes return TLS_ERR_UNSUPPORTED with a message.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.  The array exists on every GPU that loads the
+ *   library until the process exits.  All calls on a device share it and it
+ *   keeps the last call's scores (each call writes every score it reads, so
+ *   nothing needs clearing): calls whose kernels overlap on the GPU race.
+ *   Allocates nothing. */
+TLS_API tls_status tls_block_score_topk_noalloc(const tls_shape *s, const void *q, const void *meta,
+                                                const int32_t *seq_lens, int32_t *block_idx_out, void *stream);
+
 /* Bounded host wait on a cudaEvent_t: polls until the event completes or
  * timeout_ms elapses.  Returns TLS_OK, TLS_ERR_TIMEOUT, or TLS_ERR_CUDA when
  * the event reports an error.  Never blocks longer than timeout_ms (+ 1 ms). */

@@ -142,6 +142,18 @@ bool ws_layout(const tls_shape *s, bool paged, WsLayout *w) {
 
 }  // namespace
 
+namespace tls {
+tls_status set_error(tls_status st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+}  // namespace tls
+
 extern "C" {
 
 const char *tls_version(void) { return "tls 0.1 sm_100a"; }

@@ -5,7 +5,12 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "tls.h"
+
 namespace tls {
+
+// Records a printf-style message for tls_last_error() on this thread; returns st.
+tls_status set_error(tls_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
 
 constexpr int kMaxSelectKeys = 16384;  // keys held in shared memory by one selection CTA
 

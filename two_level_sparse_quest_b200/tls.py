@@ -30,7 +30,7 @@ STATUS_NAMES = {0: "TLS_OK", 1: "TLS_ERR_INVALID_ARG", 2: "TLS_ERR_UNSUPPORTED",
 
 EXPORTED = ("tls_version", "tls_last_error", "tls_workspace_size", "tls_build_block_meta", "tls_block_score_topk",
             "tls_token_score_topk", "tls_sparse_attn_decode", "tls_sparse_attn_decode_paged", "tls_offload_reset",
-            "tls_prefetch_diff", "tls_wait_event")
+            "tls_prefetch_diff", "tls_wait_event", "tls_block_score_topk_noalloc")
 
 
 class TlsShape(ctypes.Structure):
@@ -64,6 +64,7 @@ _sigs = {
     "tls_offload_reset": ([_S, _i32, _P, _P, _P], ctypes.c_int),
     "tls_prefetch_diff": ([_S, _i32, _P, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "tls_wait_event": ([_P, _i32], ctypes.c_int),
+    "tls_block_score_topk_noalloc": ([_S, _P, _P, _P, _P, _P], ctypes.c_int),
 }
 for _name, (_args, _ret) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -181,6 +182,14 @@ def tls_prefetch_diff(shape, n_slots, host_kv, cache, slot_of_block, block_of_sl
     _check(_lib.tls_prefetch_diff(ctypes.byref(shape), int(n_slots), _ptr(host_kv), _ptr(cache), _ptr(slot_of_block),
                                   _ptr(block_of_slot), _ptr(prev_block_idx), _ptr(next_block_idx), _ptr(n_new_out),
                                   _ptr(jobs_ws), _stream(stream)), "tls_prefetch_diff")
+
+
+def tls_block_score_topk_noalloc(shape, q, meta, seq_lens, block_idx_out, stream=None):
+    """Block selection without a workspace, for callers that cannot allocate
+    device memory: the scores live in a fixed array inside the library (see
+    include/tls.h for the size limit and the sharing rules)."""
+    _check(_lib.tls_block_score_topk_noalloc(ctypes.byref(shape), _ptr(q), _ptr(meta), _ptr(seq_lens),
+                                             _ptr(block_idx_out), _stream(stream)), "tls_block_score_topk_noalloc")
 
 
 def tls_wait_event(event, timeout_ms: int) -> int:
