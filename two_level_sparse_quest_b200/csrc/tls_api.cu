@@ -38,7 +38,6 @@ tls_status cuda_status(cudaError_t e, const char *what) {
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-int elt_bytes(const tls_shape *s) { return s->kv_dtype == TLS_BF16 ? 2 : 4; }
 int n_blocks_max(const tls_shape *s) { return (s->max_ctx + s->block_size - 1) / s->block_size; }
 
 int device_sms() {
@@ -121,9 +120,9 @@ tls::AttnArgs attn_args(const tls_shape *s) {
   return a;
 }
 
-// Workspace layout: [block scores | attention partials], 256-byte aligned.
+// Workspace layout: [block scores | attention partials | error word], 256-byte aligned.
 struct WsLayout {
-  size_t scores_off, scores_bytes, part_off, part_bytes, total;
+  size_t scores_off, scores_bytes, part_off, part_bytes, err_off, total;
 };
 
 bool ws_layout(const tls_shape *s, bool paged, WsLayout *w) {
@@ -136,7 +135,8 @@ bool ws_layout(const tls_shape *s, bool paged, WsLayout *w) {
   if (!tls::attn_plan(a, &p)) return false;
   w->part_off = w->scores_bytes;
   w->part_bytes = up(p.part_floats * sizeof(float));
-  w->total = w->part_off + w->part_bytes;
+  w->err_off = w->part_off + w->part_bytes;
+  w->total = w->err_off + 256;
   return true;
 }
 
@@ -272,6 +272,7 @@ static tls_status attn_common(const tls_shape *s, const void *q, const void *K, 
   a.out = out;
   a.lse = lse_out;
   a.part = reinterpret_cast<float *>(static_cast<char *>(ws) + w.part_off);
+  a.err = reinterpret_cast<int *>(static_cast<char *>(ws) + w.err_off);
   a.paged = paged;
   tls::AttnPlan p;
   if (!tls::attn_plan(a, &p)) return fail(TLS_ERR_UNSUPPORTED, "no attention plan for this shape");

@@ -22,6 +22,8 @@
 //    that unit; a merge kernel combines the partials of each head by
 //    log-sum-exp and writes out / lse.
 #include <algorithm>
+#include <cstdlib>
+#include <cstring>
 
 #include "tls_device.cuh"
 #include "tls_internal.h"
@@ -29,7 +31,7 @@
 namespace tls {
 namespace {
 
-constexpr int kTT = 32;  // tokens per tile
+constexpr int kTT = 16;  // tokens per tile (two lanes per token in QK)
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -37,42 +39,53 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-template <typename E, int D, int DV, int HG, bool VPREFIX, int W, int NS>
+template <typename E, int D, int DV, int HG, bool VPREFIX, int NS>
 struct AttnLayout {
   static constexpr int kElt = E::kBytes;
   static constexpr int RB = D * kElt;                     // K row bytes
   static constexpr int KCH = RB / 16;                     // 16-byte chunks per K row
-  static constexpr int VB = VPREFIX ? 0 : DV * kElt;      // V row bytes (0: V inside K row)
+  static constexpr int VB = VPREFIX ? 0 : DV * kElt;      // V row bytes (0: V inside the K row)
   static constexpr int VCH = VB / 16;
   static constexpr int CPL = DV / 32;                     // output channels per lane
   static constexpr int kStageBytes = kTT * (RB + VB);
   static constexpr int kWarpBytes = NS * kStageBytes + HG * D * 4 + kTT * HG * 4 + NS * kTT * 8;
+  static constexpr int kMaxSmem = 227 * 1024;
+  static constexpr int W = (kMaxSmem / kWarpBytes) < 16 ? (kMaxSmem / kWarpBytes) : 16;  // warps per CTA
   static constexpr int kSmem = W * kWarpBytes;
-  static_assert(KCH % 8 == 0, "row must be a multiple of 128 bytes for the swizzle");
-  static_assert(DV % 32 == 0, "d_v must be a multiple of 32");
+  static_assert(KCH % 8 == 0, "the row swizzle permutes groups of 8 chunks (rows of a multiple of 128 bytes)");
+  static_assert((kTT * KCH) % 32 == 0, "issue loop covers whole warps");
+  static_assert(DV % 64 == 0, "d_v must be a multiple of 64");
+  static_assert(W >= 1, "one warp's buffers must fit in shared memory");
 };
 
-template <typename E, int D, int DV, int HG, bool VPREFIX, bool PAGED, int W, int NS>
-__global__ void __launch_bounds__(W * 32, 1) attn_split_kernel(AttnArgs a, AttnPlan p) {
-  using L = AttnLayout<E, D, DV, HG, VPREFIX, W, NS>;
+// One CTA per SM; every warp streams its own contiguous range of (unit, tile)
+// work.  Two lanes share a token: lane l handles token l & 15 and the half
+// (l >> 4) of its channels in QK.
+template <typename E, int D, int DV, int HG, bool VPREFIX, bool PAGED, int NS>
+__global__ void __launch_bounds__(AttnLayout<E, D, DV, HG, VPREFIX, NS>::W * 32, 1)
+    attn_split_kernel(AttnArgs a, AttnPlan p) {
+  using L = AttnLayout<E, D, DV, HG, VPREFIX, NS>;
   using S = typename E::storage;
   constexpr int EPC = E::kEPC;
   constexpr int CPL = L::CPL;
+  constexpr int HALF = L::KCH / 2;  // QK chunks per lane
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int tr = lane & 15, hf = lane >> 4;
   unsigned char *wbase = smem + warp * L::kWarpBytes;
-  unsigned char *stage_base = wbase;                                        // NS stages
-  float *Qs = reinterpret_cast<float *>(wbase + NS * L::kStageBytes);       // [HG][D]
-  float *Ps = Qs + HG * D;                                                  // [kTT][HG]
-  long long *Off = reinterpret_cast<long long *>(Ps + kTT * HG);            // [NS][kTT]
+  float *Qs = reinterpret_cast<float *>(wbase + NS * L::kStageBytes);  // [HG][D]
+  float *Ps = Qs + HG * D;                                             // [kTT][HG]
+  long long *Off = reinterpret_cast<long long *>(Ps + kTT * HG);       // [NS][kTT] byte offsets
 
-  const int gw = blockIdx.x * W + warp;
+  grid_dependency_wait();
+  const int gw = blockIdx.x * L::W + warp;
   const int t_begin = gw * p.tiles_per_warp;
   const int t_end = min(t_begin + p.tiles_per_warp, p.total_tiles);
   if (t_begin >= t_end) return;
 
-  const S *Kb = static_cast<const S *>(a.K);
-  const S *Vb = VPREFIX ? Kb : (PAGED ? Kb : static_cast<const S *>(a.V));
+  const unsigned char *Kb = static_cast<const unsigned char *>(a.K);
+  const unsigned char *Vb = (VPREFIX || PAGED) ? Kb : static_cast<const unsigned char *>(a.V);
+  const long long v_delta = PAGED ? static_cast<long long>(a.block_size) * L::RB : 0;
   const int Gt = a.n_q_heads / a.n_kv_heads;
 
   // Gather the rows of tile t into stage st (always commits one group).
@@ -80,46 +93,46 @@ __global__ void __launch_bounds__(W * 32, 1) attn_split_kernel(AttnArgs a, AttnP
     if (t < t_end) {
       const int unit = t / p.tiles_per_group, tile = t % p.tiles_per_group;
       const int group = unit / p.n_head_chunks;
-      const int j = tile * kTT + lane;
-      long long off = -1;
-      if (j < a.k_t) {
-        const int tok = a.token_idx[static_cast<size_t>(group) * a.k_t + j];
-        if (tok >= 0 && tok < a.max_ctx) {
-          if constexpr (PAGED) {
-            const int slot = a.slot_of_block[static_cast<size_t>(group) * a.n_blocks_max + tok / a.block_size];
-            if (slot >= 0 && slot < a.n_slots)
-              off = ((static_cast<long long>(group) * a.n_slots + slot) * 2 * a.block_size + tok % a.block_size) * D;
-          } else {
-            off = (static_cast<long long>(group) * a.max_ctx + tok) * D;
+      if (lane < kTT) {
+        const int j = tile * kTT + lane;
+        long long off = -1;
+        if (j < a.k_t) {
+          const int tok = a.token_idx[static_cast<size_t>(group) * a.k_t + j];
+          if (tok >= 0 && tok < a.max_ctx) {
+            if constexpr (PAGED) {
+              const int slot = a.slot_of_block[static_cast<size_t>(group) * a.n_blocks_max + tok / a.block_size];
+              if (slot >= 0 && slot < a.n_slots)
+                off = ((static_cast<long long>(group) * a.n_slots + slot) * 2 * a.block_size + tok % a.block_size) *
+                      L::RB;
+            } else {
+              off = (static_cast<long long>(group) * a.max_ctx + tok) * L::RB;
+            }
           }
         }
+        Off[st * kTT + lane] = off;
       }
-      Off[st * kTT + lane] = off;
       __syncwarp();
-      unsigned char *Ks = stage_base + st * L::kStageBytes;
-#pragma unroll 4
-      for (int idx = lane; idx < kTT * L::KCH; idx += 32) {
+      unsigned char *Ks = wbase + st * L::kStageBytes;
+      unsigned char *Vs = Ks + kTT * L::RB;
+#pragma unroll
+      for (int i = 0; i < kTT * L::KCH / 32; ++i) {
+        const int idx = i * 32 + lane;
         const int row = idx / L::KCH, c = idx % L::KCH;
         const long long o = Off[st * kTT + row];
-        const S *src = Kb + (o >= 0 ? o : 0) + c * EPC;
-        cp_async16(Ks + row * L::RB + ((c ^ (row & 7)) * 16), src, o >= 0);
-      }
-      if constexpr (!VPREFIX) {
-        unsigned char *Vs = Ks + kTT * L::RB;
-#pragma unroll 4
-        for (int idx = lane; idx < kTT * L::VCH; idx += 32) {
-          const int row = idx / L::VCH, c = idx % L::VCH;
-          const long long o = Off[st * kTT + row];
-          const long long vo = PAGED ? o + static_cast<long long>(a.block_size) * D : o;
-          const S *src = Vb + (o >= 0 ? vo : 0) + c * EPC;
-          cp_async16(Vs + row * L::VB + c * 16, src, o >= 0);
+        const bool ok = o >= 0;
+        const long long ob = ok ? o : 0;
+        cp_async16(Ks + row * L::RB + ((c ^ (row & 7)) << 4), Kb + ob + (c << 4), ok);
+        if constexpr (!VPREFIX) {
+          // GQA: V rows have the same chunk count as K rows
+          cp_async16(Vs + row * L::VB + (c << 4), Vb + ob + v_delta + (c << 4), ok);
         }
       }
     }
     cp_async_commit();
   };
 
-  float m[HG], l[HG], acc[HG][CPL];
+  float2 acc[HG][CPL / 2];
+  float m[HG], l[HG];
   int cur_unit = -1;
 
   auto reset = [&]() {
@@ -128,23 +141,23 @@ __global__ void __launch_bounds__(W * 32, 1) attn_split_kernel(AttnArgs a, AttnP
       m[h] = -INFINITY;
       l[h] = 0.f;
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) acc[h][c] = 0.f;
+      for (int c = 0; c < CPL / 2; ++c) acc[h][c] = make_float2(0.f, 0.f);
     }
   };
 
   auto flush = [&](int unit) {
     const int first = (unit * p.tiles_per_group) / p.tiles_per_warp;
     const int piece = gw - first;
+    const size_t units = static_cast<size_t>(a.batch) * a.n_kv_heads * p.n_head_chunks;
     float *ml = a.part + (static_cast<size_t>(unit) * p.max_pieces + piece) * HG * 2;
-    float *po = a.part + static_cast<size_t>(a.batch) * a.n_kv_heads * p.n_head_chunks * p.max_pieces * HG * 2 +
-                (static_cast<size_t>(unit) * p.max_pieces + piece) * HG * DV;
+    float *po = a.part + units * p.max_pieces * HG * 2 + (static_cast<size_t>(unit) * p.max_pieces + piece) * HG * DV;
 #pragma unroll
     for (int h = 0; h < HG; ++h) {
       const float lt = warp_sum(l[h]);
       if (lane == 0) { ml[h * 2] = m[h]; ml[h * 2 + 1] = lt; }
-      float *dst = po + h * DV + lane * CPL;
+      float2 *dst = reinterpret_cast<float2 *>(po + h * DV + lane * CPL);
 #pragma unroll
-      for (int c = 0; c < CPL; c += 2) *reinterpret_cast<float2 *>(dst + c) = make_float2(acc[h][c], acc[h][c + 1]);
+      for (int c = 0; c < CPL / 2; ++c) dst[c] = acc[h][c];
     }
   };
 
@@ -171,17 +184,18 @@ __global__ void __launch_bounds__(W * 32, 1) attn_split_kernel(AttnArgs a, AttnP
       load_q(unit);
       cur_unit = unit;
     }
-    const unsigned char *Ks = stage_base + st * L::kStageBytes;
-    const bool valid = Off[st * kTT + lane] >= 0;
+    const unsigned char *Ks = wbase + st * L::kStageBytes;
+    const bool valid = Off[st * kTT + tr] >= 0;
 
-    // ---- scores: lane = token row
+    // ---- scores: token tr, channel half hf
     float2 s2[HG];
 #pragma unroll
     for (int h = 0; h < HG; ++h) s2[h] = make_float2(0.f, 0.f);
-    const unsigned char *krow = Ks + lane * L::RB;
-#pragma unroll 8
-    for (int j = 0; j < L::KCH; ++j) {
-      const uint4 kc = *reinterpret_cast<const uint4 *>(krow + ((j ^ (lane & 7)) * 16));
+    const unsigned char *krow = Ks + tr * L::RB;
+#pragma unroll 4
+    for (int jj = 0; jj < HALF; ++jj) {
+      const int j = hf * HALF + jj;
+      const uint4 kc = *reinterpret_cast<const uint4 *>(krow + ((j ^ (tr & 7)) << 4));
       float kf[EPC];
       chunk_to_f32<E>(kc, kf);
 #pragma unroll
@@ -195,21 +209,29 @@ __global__ void __launch_bounds__(W * 32, 1) attn_split_kernel(AttnArgs a, AttnP
         }
       }
     }
-    // ---- online softmax (log2 domain)
+    // ---- online softmax (log2 domain); both lanes of a token hold its score
 #pragma unroll
     for (int h = 0; h < HG; ++h) {
-      const float sc = valid ? (s2[h].x + s2[h].y) : -INFINITY;
-      const float mn = fmaxf(m[h], warp_max(sc));
+      float sc = s2[h].x + s2[h].y;
+      sc += __shfl_xor_sync(0xffffffffu, sc, 16);
+      sc = valid ? sc : -INFINITY;
+      float tm = sc;
+#pragma unroll
+      for (int o = 8; o > 0; o >>= 1) tm = fmaxf(tm, __shfl_xor_sync(0xffffffffu, tm, o));
+      const float mn = fmaxf(m[h], tm);
       float alpha = 1.f, pr = 0.f;
       if (mn != -INFINITY) {
         alpha = ex2(m[h] - mn);
         pr = ex2(sc - mn);
       }
-      l[h] = l[h] * alpha + pr;
+      l[h] = l[h] * alpha + (hf == 0 ? pr : 0.f);
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) acc[h][c] *= alpha;
+      for (int c = 0; c < CPL / 2; ++c) {
+        acc[h][c].x *= alpha;
+        acc[h][c].y *= alpha;
+      }
       m[h] = mn;
-      Ps[lane * HG + h] = pr;
+      if (hf == 0) Ps[tr * HG + h] = pr;
     }
     __syncwarp();
     // ---- o += p v: lane owns channels [lane*CPL, lane*CPL + CPL)
@@ -217,15 +239,22 @@ __global__ void __launch_bounds__(W * 32, 1) attn_split_kernel(AttnArgs a, AttnP
 #pragma unroll 4
     for (int r = 0; r < kTT; ++r) {
       float pv[HG];
+      if constexpr (HG % 4 == 0) {
 #pragma unroll
-      for (int h = 0; h < HG; ++h) pv[h] = Ps[r * HG + h];
+        for (int h = 0; h < HG; h += 4) {
+          const float4 p4 = *reinterpret_cast<const float4 *>(Ps + r * HG + h);
+          pv[h] = p4.x; pv[h + 1] = p4.y; pv[h + 2] = p4.z; pv[h + 3] = p4.w;
+        }
+      } else {
+#pragma unroll
+        for (int h = 0; h < HG; ++h) pv[h] = Ps[r * HG + h];
+      }
       float vf[CPL];
       if constexpr (VPREFIX) {
-        // channels lane*CPL.. live in K-row chunks (swizzled)
 #pragma unroll
         for (int q = 0; q < CPL / EPC; ++q) {
           const int c = lane * (CPL / EPC) + q;
-          const uint4 vc = *reinterpret_cast<const uint4 *>(Vs + r * L::RB + ((c ^ (r & 7)) * 16));
+          const uint4 vc = *reinterpret_cast<const uint4 *>(Vs + r * L::RB + ((c ^ (r & 7)) << 4));
           chunk_to_f32<E>(vc, vf + q * EPC);
         }
       } else {
@@ -247,13 +276,9 @@ __global__ void __launch_bounds__(W * 32, 1) attn_split_kernel(AttnArgs a, AttnP
       }
 #pragma unroll
       for (int h = 0; h < HG; ++h) {
+        const float2 pp = make_float2(pv[h], pv[h]);
 #pragma unroll
-        for (int c = 0; c < CPL; c += 2) {
-          float2 o2 = make_float2(acc[h][c], acc[h][c + 1]);
-          ffma2(o2, make_float2(vf[c], vf[c + 1]), make_float2(pv[h], pv[h]));
-          acc[h][c] = o2.x;
-          acc[h][c + 1] = o2.y;
-        }
+        for (int c = 0; c < CPL / 2; ++c) ffma2(acc[h][c], make_float2(vf[2 * c], vf[2 * c + 1]), pp);
       }
     }
     __syncwarp();
@@ -262,55 +287,63 @@ __global__ void __launch_bounds__(W * 32, 1) attn_split_kernel(AttnArgs a, AttnP
   cp_async_wait<0>();
 }
 
+// Log-sum-exp merge of the pieces of one (unit, head, 32-channel slice); one
+// warp each, one channel per lane.  The pieces' (max, sum) are read by the
+// lanes in parallel, 32 pieces at a time; their partial outputs are then read
+// as independent coalesced loads.
 template <int DV, int HG>
 __global__ void __launch_bounds__(128) attn_merge_kernel(AttnArgs a, AttnPlan p) {
-  constexpr int CPL = DV / 32;
+  constexpr int NSL = DV / 32;
+  grid_dependency_wait();
   const int lane = threadIdx.x & 31;
   const int w = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int n_units = a.batch * a.n_kv_heads * p.n_head_chunks;
-  if (w >= n_units * HG) return;
-  const int unit = w / HG, hh = w % HG;
+  if (w >= n_units * HG * NSL) return;
+  const int unit = w / (HG * NSL), rem = w % (HG * NSL);
+  const int hh = rem / NSL, sl = rem % NSL;
   const int group = unit / p.n_head_chunks, hc = unit % p.n_head_chunks;
   const int b = group / a.n_kv_heads, g = group % a.n_kv_heads;
   const int Gt = a.n_q_heads / a.n_kv_heads;
   const int head = g * Gt + hc * HG + hh;
   const int first = (unit * p.tiles_per_group) / p.tiles_per_warp;
   const int last = ((unit + 1) * p.tiles_per_group - 1) / p.tiles_per_warp;
+  const int n_pieces = last - first + 1;
+  const int ch = sl * 32 + lane;
   const float *ml = a.part + static_cast<size_t>(unit) * p.max_pieces * HG * 2;
   const float *po = a.part + static_cast<size_t>(n_units) * p.max_pieces * HG * 2 +
-                    static_cast<size_t>(unit) * p.max_pieces * HG * DV;
-  float M = -INFINITY;
-  for (int q = 0; q <= last - first; ++q) M = fmaxf(M, ml[(q * HG + hh) * 2]);
-  float o[CPL];
+                    static_cast<size_t>(unit) * p.max_pieces * HG * DV + hh * DV + ch;
+  float M = -INFINITY, Lsum = 0.f, o = 0.f;
+  for (int q0 = 0; q0 < n_pieces; q0 += 32) {
+    const int q = q0 + lane;
+    const float mq = q < n_pieces ? ml[(q * HG + hh) * 2] : -INFINITY;
+    const float lq = q < n_pieces ? ml[(q * HG + hh) * 2 + 1] : 0.f;
+    const float Mn = fmaxf(M, warp_max(mq));
+    if (Mn == -INFINITY) continue;
+    const float scale_old = ex2(M - Mn);
+    const float wq = ex2(mq - Mn);
+    Lsum = Lsum * scale_old + warp_sum(wq * lq);
+    o *= scale_old;
+    const int nq = min(32, n_pieces - q0);
+    float v[32];
 #pragma unroll
-  for (int c = 0; c < CPL; ++c) o[c] = 0.f;
-  float Lsum = 0.f;
-  if (M != -INFINITY) {
-    for (int q = 0; q <= last - first; ++q) {
-      const float wq = ex2(ml[(q * HG + hh) * 2] - M);
-      Lsum += wq * ml[(q * HG + hh) * 2 + 1];
-      const float *src = po + (static_cast<size_t>(q) * HG + hh) * DV;
+    for (int k = 0; k < 32; ++k) v[k] = k < nq ? po[static_cast<size_t>(q0 + k) * HG * DV] : 0.f;
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) o[c] += wq * src[c * 32 + lane];
-    }
+    for (int k = 0; k < 32; ++k) o = fmaf(__shfl_sync(0xffffffffu, wq, k), v[k], o);
+    M = Mn;
   }
-  const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-  const size_t ob = (static_cast<size_t>(b) * a.n_q_heads + head) * DV;
-#pragma unroll
-  for (int c = 0; c < CPL; ++c) {
-    const float v = o[c] * inv;
-    if (a.out_dtype == 1) static_cast<uint16_t *>(a.out)[ob + c * 32 + lane] = f32_to_bf16_rne(v);
-    else static_cast<float *>(a.out)[ob + c * 32 + lane] = v;
-  }
-  if (a.lse && lane == 0)
+  const float res = Lsum > 0.f ? o / Lsum : 0.f;
+  const size_t ob = (static_cast<size_t>(b) * a.n_q_heads + head) * DV + ch;
+  if (a.out_dtype == 1) static_cast<uint16_t *>(a.out)[ob] = f32_to_bf16_rne(res);
+  else static_cast<float *>(a.out)[ob] = res;
+  if (a.lse && sl == 0 && lane == 0)
     a.lse[static_cast<size_t>(b) * a.n_q_heads + head] =
         (M == -INFINITY || Lsum <= 0.f) ? -INFINITY : (M + log2f(Lsum)) * 0.69314718055994531f;
 }
 
-template <typename E, int D, int DV, int HG, bool VPREFIX, bool PAGED, int W, int NS>
+template <typename E, int D, int DV, int HG, bool VPREFIX, bool PAGED, int NS>
 cudaError_t run_attention(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) {
-  using L = AttnLayout<E, D, DV, HG, VPREFIX, W, NS>;
-  auto kern = attn_split_kernel<E, D, DV, HG, VPREFIX, PAGED, W, NS>;
+  using L = AttnLayout<E, D, DV, HG, VPREFIX, NS>;
+  auto kern = attn_split_kernel<E, D, DV, HG, VPREFIX, PAGED, NS>;
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -319,53 +352,85 @@ cudaError_t run_attention(const AttnArgs &a, const AttnPlan &p, cudaStream_t st)
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  kern<<<p.grid, W * 32, L::kSmem, st>>>(a, p);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  const int n_warps = a.batch * a.n_kv_heads * p.n_head_chunks * HG;
-  attn_merge_kernel<DV, HG><<<(n_warps + 3) / 4, 128, 0, st>>>(a, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(p.grid), dim3(L::W * 32), L::kSmem, st, a, p);
+}
+
+template <int DV, int HG>
+cudaError_t run_merge(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) {
+  const int n_warps = a.batch * a.n_kv_heads * p.n_head_chunks * HG * (DV / 32);
+  return launch_pdl(attn_merge_kernel<DV, HG>, dim3((n_warps + 3) / 4), dim3(128), 0, st, a, p);
 }
 
 // Kernel-set selection.  Returns false for shapes outside the compiled set.
 struct Variant {
-  int warps, stages, head_chunk;
+  int warps, head_chunk;
 };
+
+constexpr int kStages = 3;
+
+template <typename E, int D, int DV, int HG, bool VPREFIX>
+constexpr int warps_of() {
+  return AttnLayout<E, D, DV, HG, VPREFIX, kStages>::W;
+}
+
+template <typename E, int D>
+int gqa_warps(int G) {
+  switch (G) {
+    case 1: return warps_of<E, D, D, 1, false>();
+    case 2: return warps_of<E, D, D, 2, false>();
+    case 4: return warps_of<E, D, D, 4, false>();
+    default: return warps_of<E, D, D, 8, false>();
+  }
+}
 
 bool pick_variant(const AttnArgs &a, Variant *v) {
   const int G = a.n_q_heads / a.n_kv_heads;
   if (a.v_is_k_prefix) {
     if (a.dtype != 1 || a.d_qk != 576 || a.d_v != 512 || a.paged) return false;
     if (G % 4 != 0 || G > 128) return false;
-    *v = {2, 2, 4};
+    *v = {warps_of<BF16, 576, 512, 4, true>(), 4};
     return true;
   }
   if (a.d_qk != a.d_v || (a.d_qk != 64 && a.d_qk != 128)) return false;
   if (G != 1 && G != 2 && G != 4 && G != 8) return false;
-  const int rb = a.d_qk * (a.dtype == 1 ? 2 : 4);
-  if (rb == 128) *v = {8, 3, G};
-  else if (rb == 256) *v = {4, 3, G};
-  else *v = {3, 2, G};
+  int w;
+  if (a.dtype == 1) w = a.d_qk == 128 ? gqa_warps<BF16, 128>(G) : gqa_warps<BF16, 64>(G);
+  else w = a.d_qk == 128 ? gqa_warps<F32, 128>(G) : gqa_warps<F32, 64>(G);
+  *v = {w, G};
   return true;
 }
 
 template <typename E, int D, bool PAGED>
 cudaError_t dispatch_gqa(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) {
-  constexpr int RB = D * E::kBytes;
-  constexpr int W = RB == 128 ? 8 : (RB == 256 ? 4 : 3);
-  constexpr int NS = RB == 512 ? 2 : 3;
   switch (p.head_chunk) {
-    case 1: return run_attention<E, D, D, 1, false, PAGED, W, NS>(a, p, st);
-    case 2: return run_attention<E, D, D, 2, false, PAGED, W, NS>(a, p, st);
-    case 4: return run_attention<E, D, D, 4, false, PAGED, W, NS>(a, p, st);
-    case 8: return run_attention<E, D, D, 8, false, PAGED, W, NS>(a, p, st);
+    case 1: return run_attention<E, D, D, 1, false, PAGED, kStages>(a, p, st);
+    case 2: return run_attention<E, D, D, 2, false, PAGED, kStages>(a, p, st);
+    case 4: return run_attention<E, D, D, 4, false, PAGED, kStages>(a, p, st);
+    case 8: return run_attention<E, D, D, 8, false, PAGED, kStages>(a, p, st);
   }
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
+// GQA bf16 d = 128 has two kernels: the CUDA-core one (default; faster on the
+// 96k decode workload, where the gather is the bound) and the tcgen05 one
+// (TLS_ATTN_IMPL=tensor_core; read once per process).
+static bool tensor_core_allowed() {
+  static int allowed = -1;
+  if (allowed < 0) {
+    const char *e = getenv("TLS_ATTN_IMPL");
+    allowed = (e && strcmp(e, "tensor_core") == 0) ? 1 : 0;
+  }
+  return allowed == 1;
+}
+
 bool attn_plan(const AttnArgs &a, AttnPlan *p) {
+  if (tensor_core_allowed() && attn_tc_supported(a)) {
+    p->tensor_core = 1;
+    return attn_tc_plan(a, p);
+  }
+  p->tensor_core = 0;
   Variant v;
   if (!pick_variant(a, &v)) return false;
   const int G = a.n_q_heads / a.n_kv_heads;
@@ -387,14 +452,33 @@ bool attn_plan(const AttnArgs &a, AttnPlan *p) {
   return true;
 }
 
-cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) {
-  if (a.v_is_k_prefix) return run_attention<BF16, 576, 512, 4, true, false, 2, 2>(a, p, st);
+static cudaError_t launch_split(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) {
+  if (p.tensor_core) return launch_attention_tc(a, p, st);
+  if (a.v_is_k_prefix) return run_attention<BF16, 576, 512, 4, true, false, kStages>(a, p, st);
   if (a.dtype == 1) {
     if (a.d_qk == 128) return a.paged ? dispatch_gqa<BF16, 128, true>(a, p, st) : dispatch_gqa<BF16, 128, false>(a, p, st);
     return a.paged ? dispatch_gqa<BF16, 64, true>(a, p, st) : dispatch_gqa<BF16, 64, false>(a, p, st);
   }
   if (a.d_qk == 128) return a.paged ? dispatch_gqa<F32, 128, true>(a, p, st) : dispatch_gqa<F32, 128, false>(a, p, st);
   return a.paged ? dispatch_gqa<F32, 64, true>(a, p, st) : dispatch_gqa<F32, 64, false>(a, p, st);
+}
+
+cudaError_t launch_attention_merge(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) {
+  if (a.v_is_k_prefix) return run_merge<512, 4>(a, p, st);
+  const int dv = a.d_v;
+  switch (p.head_chunk) {
+    case 1: return dv == 128 ? run_merge<128, 1>(a, p, st) : run_merge<64, 1>(a, p, st);
+    case 2: return dv == 128 ? run_merge<128, 2>(a, p, st) : run_merge<64, 2>(a, p, st);
+    case 4: return dv == 128 ? run_merge<128, 4>(a, p, st) : run_merge<64, 4>(a, p, st);
+    case 8: return dv == 128 ? run_merge<128, 8>(a, p, st) : run_merge<64, 8>(a, p, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) {
+  cudaError_t e = launch_split(a, p, st);
+  if (e != cudaSuccess) return e;
+  return launch_attention_merge(a, p, st);
 }
 
 }  // namespace tls

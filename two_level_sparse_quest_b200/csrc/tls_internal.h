@@ -9,6 +9,25 @@
 
 namespace tls {
 
+// Launch with programmatic dependent launch enabled: the kernel's launch and
+// its pre-wait prologue overlap the tail of the previous kernel in the stream
+// (the kernel itself waits for that grid before touching global memory).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Records a printf-style message for tls_last_error() on this thread; returns st.
 tls_status set_error(tls_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
 
@@ -33,6 +52,7 @@ struct BlockScoreArgs {
   int32_t *block_idx; // [B*H_kv][k_b]
   int batch, n_q_heads, n_kv_heads, d, block_size, n_blocks_max, max_ctx, k_b, dtype;
   int num_sms;
+  int *err;  // optional: set to 1 when a bounded wait gave up
 };
 cudaError_t launch_block_score(const BlockScoreArgs &a, cudaStream_t st);
 cudaError_t launch_block_topk(const BlockScoreArgs &a, cudaStream_t st);
@@ -59,6 +79,7 @@ struct AttnArgs {
   void *out;
   float *lse;
   float *part;  // workspace partials
+  int *err;     // workspace word: set to 1 when a bounded wait in a kernel gave up
   int batch, n_q_heads, n_kv_heads, d_qk, d_v, v_is_k_prefix, block_size, n_blocks_max, max_ctx, k_t;
   int dtype, out_dtype, paged;
   float scale_log2;  // softmax_scale * log2(e)
@@ -67,12 +88,19 @@ struct AttnArgs {
 // Partial-result layout chosen for a shape on a device; shared by the
 // workspace query and the launch so both agree.
 struct AttnPlan {
+  int tensor_core;  // 1: tcgen05 kernel (tiles_per_warp counts tiles per CTA)
   int warps_per_cta, tokens_per_tile, head_chunk, n_head_chunks;
   int tiles_per_group, total_tiles, grid, tiles_per_warp, max_pieces;
   size_t part_floats;  // floats of workspace for partials
 };
 bool attn_plan(const AttnArgs &a, AttnPlan *p);
 cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &p, cudaStream_t st);
+// tensor-core (tcgen05) attention for GQA bf16 d = 128
+bool attn_tc_supported(const AttnArgs &a);
+bool attn_tc_plan(const AttnArgs &a, AttnPlan *p);
+cudaError_t launch_attention_tc(const AttnArgs &a, const AttnPlan &p, cudaStream_t st);
+// merge kernel of the partials (shared by both attention paths)
+cudaError_t launch_attention_merge(const AttnArgs &a, const AttnPlan &p, cudaStream_t st);
 
 struct OffloadArgs {
   const void *host_kv;  // device-visible pointer of the pinned host KV

@@ -15,6 +15,7 @@ namespace {
 
 template <typename E>
 __global__ void __launch_bounds__(256) build_meta_kernel(MetaArgs a) {
+  grid_dependency_wait();
   constexpr int EPC = E::kEPC;
   const int chunks = a.d / EPC;  // 16-byte chunks per key row
   const int group = blockIdx.y;  // b * H_kv + g
@@ -55,6 +56,7 @@ __global__ void __launch_bounds__(256) build_meta_kernel(MetaArgs a) {
 
 template <typename E>
 __global__ void __launch_bounds__(256) build_slab_kernel(MetaArgs a) {
+  grid_dependency_wait();
   using S = typename E::storage;
   const int group = blockIdx.y;
   const int b = group / a.n_kv_heads;
@@ -74,17 +76,15 @@ cudaError_t launch_build_meta(const MetaArgs &a, cudaStream_t st) {
   const int epc = a.dtype == 1 ? BF16::kEPC : F32::kEPC;
   const long long items = static_cast<long long>(a.n_blocks_max) * (a.d / epc);
   dim3 grid(static_cast<unsigned>((items + 255) / 256), a.batch * a.n_kv_heads);
-  if (a.dtype == 1) build_meta_kernel<BF16><<<grid, 256, 0, st>>>(a);
-  else build_meta_kernel<F32><<<grid, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  if (a.dtype == 1) return launch_pdl(build_meta_kernel<BF16>, grid, dim3(256), 0, st, a);
+  return launch_pdl(build_meta_kernel<F32>, grid, dim3(256), 0, st, a);
 }
 
 cudaError_t launch_build_slab(const MetaArgs &a, cudaStream_t st) {
   const long long items = static_cast<long long>(a.max_ctx) * a.n_label;
   dim3 grid(static_cast<unsigned>((items + 255) / 256), a.batch * a.n_kv_heads);
-  if (a.dtype == 1) build_slab_kernel<BF16><<<grid, 256, 0, st>>>(a);
-  else build_slab_kernel<F32><<<grid, 256, 0, st>>>(a);
-  return cudaGetLastError();
+  if (a.dtype == 1) return launch_pdl(build_slab_kernel<BF16>, grid, dim3(256), 0, st, a);
+  return launch_pdl(build_slab_kernel<F32>, grid, dim3(256), 0, st, a);
 }
 
 }  // namespace tls

@@ -24,6 +24,7 @@ constexpr int kMaxBitmapWords = 16384 / 32;
 constexpr int kMaxSlots = 4096;
 
 __global__ void fill_neg1_kernel(int32_t *p, size_t n) {
+  grid_dependency_wait();
   for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x)
     p[i] = -1;
@@ -33,6 +34,7 @@ __global__ void __launch_bounds__(kDiffThreads) prefetch_diff_kernel(OffloadArgs
   __shared__ uint32_t keep[kMaxBitmapWords];
   __shared__ int16_t free_list[kMaxSlots];
   __shared__ int sh[33];
+  grid_dependency_wait();
   const int group = blockIdx.x;
   const int nbm = a.n_blocks_max;
   int32_t *sob = a.slot_of_block + static_cast<size_t>(group) * nbm;
@@ -106,6 +108,7 @@ __global__ void __launch_bounds__(kDiffThreads) prefetch_diff_kernel(OffloadArgs
 
 // One CTA per (job, group); a job is one block of 2 * bs * d elements.
 __global__ void __launch_bounds__(256) copy_blocks_kernel(OffloadArgs a, int block_bytes) {
+  grid_dependency_wait();
   const int group = blockIdx.y, q = blockIdx.x;
   if (q >= a.n_new[group]) return;
   const int32_t *jobs = a.jobs + static_cast<size_t>(group) * a.k_b * 2;
@@ -134,21 +137,17 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(OffloadArgs a, int blo
 
 cudaError_t launch_offload_reset(const OffloadArgs &a, cudaStream_t st) {
   const size_t groups = static_cast<size_t>(a.batch) * a.n_kv_heads;
-  fill_neg1_kernel<<<256, 256, 0, st>>>(a.slot_of_block, groups * a.n_blocks_max);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(fill_neg1_kernel, dim3(256), dim3(256), 0, st, a.slot_of_block, groups * a.n_blocks_max);
   if (e != cudaSuccess) return e;
-  fill_neg1_kernel<<<64, 256, 0, st>>>(a.block_of_slot, groups * a.n_slots);
-  return cudaGetLastError();
+  return launch_pdl(fill_neg1_kernel, dim3(64), dim3(256), 0, st, a.block_of_slot, groups * a.n_slots);
 }
 
 cudaError_t launch_prefetch_diff(const OffloadArgs &a, cudaStream_t st) {
   const int groups = a.batch * a.n_kv_heads;
-  prefetch_diff_kernel<<<groups, kDiffThreads, 0, st>>>(a);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(prefetch_diff_kernel, dim3(groups), dim3(kDiffThreads), 0, st, a);
   if (e != cudaSuccess) return e;
   const int block_bytes = 2 * a.block_size * a.d * (a.dtype == 1 ? 2 : 4);
-  copy_blocks_kernel<<<dim3(a.k_b, groups), 256, 0, st>>>(a, block_bytes);
-  return cudaGetLastError();
+  return launch_pdl(copy_blocks_kernel, dim3(a.k_b, groups), dim3(256), 0, st, a, block_bytes);
 }
 
 }  // namespace tls

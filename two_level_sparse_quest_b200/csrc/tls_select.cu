@@ -16,6 +16,8 @@
 // 2.A.2): one CTA per group gathers the label-channel slab rows of the
 // candidate tokens (a block's rows are contiguous), scores them against
 // Qbar_L = sum_h q_h[L] in fp32, keeps the keys in shared memory and selects.
+#include <algorithm>
+
 #include "tls_device.cuh"
 #include "tls_internal.h"
 
@@ -23,9 +25,12 @@ namespace tls {
 namespace {
 
 constexpr int kScoreThreads = 256;
-constexpr int kScoreUnroll = 4;
+constexpr int kScoreCtasPerSm = 4;
 
-// NCH: 16-byte chunks per summary row (2 * d * bytes / 16).
+// NCH: 16-byte chunks per summary row (2 * d * bytes / 16).  grid.y = group,
+// grid.x = a contiguous slice of the group's rows.  A warp owns whole rows
+// (16-byte chunk per lane, non-allocating loads); the first rows' loads are
+// issued before the head fold so that the query reads overlap them.
 template <typename E, int NCH>
 __global__ void __launch_bounds__(kScoreThreads) block_score_kernel(BlockScoreArgs a, int rows_per_cta) {
   constexpr int EPC = E::kEPC;
@@ -33,43 +38,26 @@ __global__ void __launch_bounds__(kScoreThreads) block_score_kernel(BlockScoreAr
   constexpr int RPW = 32 / LPR;                       // rows per warp step
   constexpr int CPL = (NCH + 31) / 32;                // chunks per lane
   constexpr int NWARP = kScoreThreads / 32;
+  constexpr int STEP = NWARP * RPW;
+  constexpr int U = CPL >= 4 ? 2 : 4;                 // rows in flight per warp (per lane: U * CPL loads)
   extern __shared__ float qpm[];                      // [2d]: Q^+ then Q^-
   const int group = blockIdx.y;
   const int b = group / a.n_kv_heads, g = group % a.n_kv_heads;
   const int G = a.n_q_heads / a.n_kv_heads;
   const int d = a.d;
-  const int seq = min(max(a.seq_lens[b], 0), a.max_ctx);
-  const int nb = (seq + a.block_size - 1) / a.block_size;
-  // Fold the group's heads into the sign-split query.
-  for (int i = threadIdx.x; i < d; i += kScoreThreads) {
-    float pos = 0.f, neg = 0.f;
-    for (int hh = 0; hh < G; ++hh) {
-      float v = load_elem<E>(a.q, (static_cast<size_t>(b) * a.n_q_heads + g * G + hh) * d + i);
-      pos += fmaxf(v, 0.f);
-      neg += fminf(v, 0.f);
-    }
-    qpm[i] = pos;
-    qpm[d + i] = neg;
-  }
-  __syncthreads();
+  const int nbm = a.n_blocks_max;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int sub = lane / LPR, cl = lane % LPR;  // row within the warp step, chunk lane
-  float qr[CPL][EPC];
-#pragma unroll
-  for (int j = 0; j < CPL; ++j) {
-    const int c = cl + j * 32;
-#pragma unroll
-    for (int e = 0; e < EPC; ++e) qr[j][e] = (c < NCH) ? qpm[c * EPC + e] : 0.f;
-  }
+  grid_dependency_wait();
+  const int sq = min(max(a.seq_lens[b], 0), a.max_ctx);
+  const int nb = (sq + a.block_size - 1) / a.block_size;
   const int r0 = blockIdx.x * rows_per_cta;
-  const int r1 = min(r0 + rows_per_cta, a.n_blocks_max);
-  const char *meta = static_cast<const char *>(a.meta) + static_cast<size_t>(group) * a.n_blocks_max * (NCH * 16);
-  float *out = a.scores + static_cast<size_t>(group) * a.n_blocks_max;
-  constexpr int STEP = NWARP * RPW;
-  for (int rb = r0 + warp * RPW; rb < r1; rb += STEP * kScoreUnroll) {
-    uint4 v[kScoreUnroll][CPL];
+  const int r1 = min(r0 + rows_per_cta, nbm);
+  const char *meta = static_cast<const char *>(a.meta) + static_cast<size_t>(group) * nbm * (NCH * 16);
+  float *out = a.scores + static_cast<size_t>(group) * nbm;
+  auto load_rows = [&](int rb, uint4 (&v)[U][CPL]) {
 #pragma unroll
-    for (int u = 0; u < kScoreUnroll; ++u) {
+    for (int u = 0; u < U; ++u) {
       const int row = rb + u * STEP + sub;
       const bool ok = row < r1 && row < nb;
 #pragma unroll
@@ -79,8 +67,34 @@ __global__ void __launch_bounds__(kScoreThreads) block_score_kernel(BlockScoreAr
                                   : make_uint4(0, 0, 0, 0);
       }
     }
+  };
+  uint4 v[U][CPL];
+  int rb = r0 + warp * RPW;
+  load_rows(rb, v);  // in flight while the query is folded
+  for (int i = threadIdx.x; i < d; i += kScoreThreads) {
+    float pos = 0.f, neg = 0.f;
+    for (int hh = 0; hh < G; ++hh) {
+      const float x = load_elem<E>(a.q, (static_cast<size_t>(b) * a.n_q_heads + g * G + hh) * d + i);
+      pos += fmaxf(x, 0.f);
+      neg += fminf(x, 0.f);
+    }
+    qpm[i] = pos;
+    qpm[d + i] = neg;
+  }
+  __syncthreads();
+  float qr[CPL][EPC];
 #pragma unroll
-    for (int u = 0; u < kScoreUnroll; ++u) {
+  for (int j = 0; j < CPL; ++j) {
+    const int c = cl + j * 32;
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) qr[j][e] = (c < NCH) ? qpm[c * EPC + e] : 0.f;
+  }
+  for (; rb < r1; rb += STEP * U) {
+    uint4 nv[U][CPL];
+    const bool more = rb + STEP * U < r1;
+    if (more) load_rows(rb + STEP * U, nv);  // next rows in flight during this batch's math
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
       float acc = 0.f;
 #pragma unroll
       for (int j = 0; j < CPL; ++j) {
@@ -94,31 +108,45 @@ __global__ void __launch_bounds__(kScoreThreads) block_score_kernel(BlockScoreAr
       const int row = rb + u * STEP + sub;
       if (cl == 0 && row < r1) out[row] = (row < nb) ? acc : -INFINITY;
     }
+    if (more) {
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int j = 0; j < CPL; ++j) v[u][j] = nv[u][j];
+    }
   }
 }
 
-constexpr int kTopkThreads = 1024;
+constexpr int kTopkThreads = 512;
 
 __global__ void __launch_bounds__(kTopkThreads) block_topk_kernel(BlockScoreArgs a) {
-  extern __shared__ uint32_t keys[];
-  __shared__ int hist[256];
-  __shared__ int sh[33];
-  __shared__ int bc[2];
+  extern __shared__ uint32_t dyn[];  // keys[n_blocks_max], list[n_blocks_max]
+  __shared__ SelectSmem S;
+  uint32_t *keys = dyn;
+  uint32_t *list = dyn + a.n_blocks_max;
+  grid_dependency_wait();
   const int group = blockIdx.x;
   const int b = group / a.n_kv_heads;
   const int seq = min(max(a.seq_lens[b], 0), a.max_ctx);
   const int nb = (seq + a.block_size - 1) / a.block_size;
   const float *sc = a.scores + static_cast<size_t>(group) * a.n_blocks_max;
-  for (int i = threadIdx.x; i < nb; i += kTopkThreads) keys[i] = score_key(sc[i]);
-  __syncthreads();
   int32_t *out = a.block_idx + static_cast<size_t>(group) * a.k_b;
   const int k = min(a.k_b, nb);
   if (k <= 0) {
     for (int i = threadIdx.x; i < a.k_b; i += kTopkThreads) out[i] = -1;
     return;
   }
-  SelectResult r = block_radix_select<kTopkThreads>(keys, nb, k, hist, bc);
-  block_ordered_compact<kTopkThreads>(keys, nb, r, k, out, a.k_b, [](int i) { return i; }, sh);
+  hist_clear<kTopkThreads>(S.hist);
+  __syncthreads();
+  for (int base = 0; base < nb; base += kTopkThreads) {
+    const int i = base + threadIdx.x;
+    const bool valid = i < nb;
+    const uint32_t key = valid ? score_key(sc[i]) : 0u;
+    if (valid) keys[i] = key;
+    hist_add(S.hist, key, valid);
+  }
+  const SelectResult r = select_kth<kTopkThreads>(keys, nb, k, list, S);
+  ordered_compact<kTopkThreads>(keys, nb, r, k, out, a.k_b, [](int i) { return i; }, S);
 }
 
 // RCH: 16-byte chunks per slab row (r * bytes / 16), 1..8.
@@ -126,21 +154,26 @@ constexpr int kTokThreads = 512;
 
 template <typename E, int RCH>
 __global__ void __launch_bounds__(kTokThreads) token_topk_kernel(TokenArgs a) {
-  using S = typename E::storage;
+  using S_t = typename E::storage;
   constexpr int EPC = E::kEPC;
   // candidates whose slab rows a thread loads before scoring them
-  constexpr int kTokBatch = RCH <= 2 ? 4 : (RCH <= 4 ? 2 : 1);
-  extern __shared__ uint32_t keys[];  // [k_b * bs]
+  constexpr int kTokBatch = RCH <= 2 ? 8 : (RCH <= 4 ? 4 : 1);
+  extern __shared__ uint32_t dyn[];  // keys[C], list[C]
   __shared__ int blk[1024];
   __shared__ float qbar[64];
-  __shared__ int hist[256];
-  __shared__ int sh[33];
-  __shared__ int bc[2];
+  __shared__ SelectSmem S;
+  grid_dependency_wait();
   const int group = blockIdx.x;
   const int b = group / a.n_kv_heads, g = group % a.n_kv_heads;
   const int G = a.n_q_heads / a.n_kv_heads;
   const int seq = min(max(a.seq_lens[b], 0), a.max_ctx);
   const int bs = a.block_size, r = a.n_label;
+  const int C = a.k_b * bs;
+  const bool bs_pow2 = (bs & (bs - 1)) == 0;
+  const int bs_shift = __ffs(bs) - 1;
+  auto blk_of = [&](int j) { return bs_pow2 ? (j >> bs_shift) : (j / bs); };
+  uint32_t *keys = dyn;
+  uint32_t *list = dyn + C;
   for (int i = threadIdx.x; i < a.k_b; i += kTokThreads) {
     int v = a.block_idx[static_cast<size_t>(group) * a.k_b + i];
     blk[i] = (v >= 0 && v < a.n_blocks_max) ? v : -1;
@@ -153,12 +186,12 @@ __global__ void __launch_bounds__(kTokThreads) token_topk_kernel(TokenArgs a) {
         s += load_elem<E>(a.q, (static_cast<size_t>(b) * a.n_q_heads + g * G + hh) * a.d + ch);
     qbar[c] = s;
   }
+  hist_clear<kTokThreads>(S.hist);
   __syncthreads();
   float ql[RCH * EPC];
 #pragma unroll
   for (int e = 0; e < RCH * EPC; ++e) ql[e] = qbar[e];  // r == RCH * EPC
-  const int C = a.k_b * bs;
-  const S *slab = static_cast<const S *>(a.slab) + static_cast<size_t>(group) * a.max_ctx * r;
+  const S_t *slab = static_cast<const S_t *>(a.slab) + static_cast<size_t>(group) * a.max_ctx * r;
   float *score_out = a.token_score ? a.token_score + static_cast<size_t>(group) * C : nullptr;
   int n_valid = 0;
   for (int base = 0; base < C; base += kTokThreads * kTokBatch) {
@@ -169,8 +202,9 @@ __global__ void __launch_bounds__(kTokThreads) token_topk_kernel(TokenArgs a) {
       const int j = base + u * kTokThreads + threadIdx.x;
       int t = -1;
       if (j < C) {
-        const int bl = blk[j / bs];
-        t = bl * bs + j % bs;
+        const int jb = blk_of(j);
+        const int bl = blk[jb];
+        t = bl * bs + (j - jb * bs);
         if (bl < 0 || t >= seq) t = -1;
       }
       tok[u] = t;
@@ -181,7 +215,6 @@ __global__ void __launch_bounds__(kTokThreads) token_topk_kernel(TokenArgs a) {
 #pragma unroll
     for (int u = 0; u < kTokBatch; ++u) {
       const int j = base + u * kTokThreads + threadIdx.x;
-      if (j >= C) continue;
       float acc = 0.f;
 #pragma unroll
       for (int c = 0; c < RCH; ++c) {
@@ -191,53 +224,55 @@ __global__ void __launch_bounds__(kTokThreads) token_topk_kernel(TokenArgs a) {
         for (int e = 0; e < EPC; ++e) acc = fmaf(ql[c * EPC + e], f[e], acc);
       }
       const bool ok = tok[u] >= 0;
-      keys[j] = ok ? score_key(acc) : 0u;
+      const uint32_t key = ok ? score_key(acc) : 0u;
+      if (j < C) {
+        keys[j] = key;
+        if (score_out) score_out[j] = ok ? acc : -INFINITY;
+      }
       n_valid += ok;
-      if (score_out) score_out[j] = ok ? acc : -INFINITY;
+      hist_add(S.hist, key, ok);
     }
   }
   int total;
-  block_excl_scan<kTokThreads>(n_valid, sh, total);  // also a barrier for keys[]
+  block_excl_scan<kTokThreads>(n_valid, S.sh, total);  // also a barrier for keys[] and the histogram
   int32_t *out = a.token_idx + static_cast<size_t>(group) * a.k_t;
   const int k = min(a.k_t, total);
   if (k <= 0) {
     for (int i = threadIdx.x; i < a.k_t; i += kTokThreads) out[i] = -1;
     return;
   }
-  SelectResult res = block_radix_select<kTokThreads>(keys, C, k, hist, bc);
-  block_ordered_compact<kTokThreads>(
-      keys, C, res, k, out, a.k_t, [&](int j) { return blk[j / bs] * bs + j % bs; }, sh);
+  const SelectResult res = select_kth<kTokThreads>(keys, C, k, list, S);
+  ordered_compact<kTokThreads>(
+      keys, C, res, k, out, a.k_t, [&](int j) { const int jb = blk_of(j); return blk[jb] * bs + (j - jb * bs); }, S);
 }
 
 template <typename E, int NCH>
 cudaError_t run_block_score(const BlockScoreArgs &a, cudaStream_t st) {
+  // Several CTAs per SM; rows split evenly over each group's CTAs.
   const int groups = a.batch * a.n_kv_heads;
-  // Enough CTAs to cover every SM several times; rows split evenly per group.
-  const int want = 4 * a.num_sms;
+  const int want = kScoreCtasPerSm * a.num_sms;
   int splits = (want + groups - 1) / groups;
   const int min_rows = 8 * (kScoreThreads / 32);
-  splits = max(1, min(splits, (a.n_blocks_max + min_rows - 1) / min_rows));
+  splits = std::max(1, std::min(splits, (a.n_blocks_max + min_rows - 1) / min_rows));
   const int rows = (a.n_blocks_max + splits - 1) / splits;
   splits = (a.n_blocks_max + rows - 1) / rows;
-  dim3 grid(splits, groups);
-  block_score_kernel<E, NCH><<<grid, kScoreThreads, 2 * a.d * sizeof(float), st>>>(a, rows);
-  return cudaGetLastError();
+  return launch_pdl(block_score_kernel<E, NCH>, dim3(splits, groups), dim3(kScoreThreads), 2 * a.d * sizeof(float),
+                    st, a, rows);
 }
 
 template <typename E, int RCH>
 cudaError_t run_token_topk(const TokenArgs &a, cudaStream_t st) {
-  const size_t smem = static_cast<size_t>(a.k_b) * a.block_size * sizeof(uint32_t);
+  const size_t smem = 2 * static_cast<size_t>(a.k_b) * a.block_size * sizeof(uint32_t);
   static bool configured[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
     cudaError_t e = cudaFuncSetAttribute(token_topk_kernel<E, RCH>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kMaxSelectKeys * static_cast<int>(sizeof(uint32_t)));
+                                         2 * kMaxSelectKeys * static_cast<int>(sizeof(uint32_t)));
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  token_topk_kernel<E, RCH><<<a.batch * a.n_kv_heads, kTokThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(token_topk_kernel<E, RCH>, dim3(a.batch * a.n_kv_heads), dim3(kTokThreads), smem, st, a);
 }
 
 }  // namespace
@@ -265,13 +300,12 @@ cudaError_t launch_block_topk(const BlockScoreArgs &a, cudaStream_t st) {
   cudaGetDevice(&dev);
   if (dev < 64 && !configured[dev]) {
     cudaError_t e = cudaFuncSetAttribute(block_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kMaxSelectKeys * static_cast<int>(sizeof(uint32_t)));
+                                         2 * kMaxSelectKeys * static_cast<int>(sizeof(uint32_t)));
     if (e != cudaSuccess) return e;
     configured[dev] = true;
   }
-  const size_t smem = static_cast<size_t>(a.n_blocks_max) * sizeof(uint32_t);
-  block_topk_kernel<<<a.batch * a.n_kv_heads, kTopkThreads, smem, st>>>(a);
-  return cudaGetLastError();
+  const size_t smem = 2 * static_cast<size_t>(a.n_blocks_max) * sizeof(uint32_t);
+  return launch_pdl(block_topk_kernel, dim3(a.batch * a.n_kv_heads), dim3(kTopkThreads), smem, st, a);
 }
 
 cudaError_t launch_token_topk(const TokenArgs &a, cudaStream_t st) {
