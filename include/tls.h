@@ -99,10 +99,11 @@ TLS_API const char *tls_version(void);
 /* Message of the last failed call on this thread ("" if none). */
 TLS_API const char *tls_last_error(void);
 
-/* Bytes of device workspace that tls_block_score_topk, tls_token_score_topk and
- * tls_sparse_attn_decode(_paged) need for this shape on the current device.
- * One buffer of this size serves all three; calls that run concurrently need
- * separate buffers.  Returns 0 for an invalid shape (see tls_last_error). */
+/* Bytes of device workspace that tls_sparse_attn_decode(_paged) need for this
+ * shape on the current device (the split-KV partials).  Calls that run
+ * concurrently need separate buffers.  The selection stages take a workspace
+ * argument too but use none (their keys stay in on-chip memory); they accept
+ * NULL.  Returns 0 for an invalid shape (see tls_last_error). */
 TLS_API size_t tls_workspace_size(const tls_shape *s);
 
 /* Set-up: block summary and label-channel slab of a KV cache.
@@ -134,7 +135,9 @@ TLS_API tls_status tls_build_block_meta(const tls_shape *s, const void *K, const
  *   block_idx_out  device int32 [B][H_kv][k_b], ascending block ids, -1 padded
  *   block_score_out device fp32 [B][H_kv][ceil(max_ctx/bs)] or NULL; blocks at or
  *                  beyond ceil(seq_len/bs) hold -inf
- *   ws, ws_bytes   device workspace of at least tls_workspace_size(s) bytes */
+ *   ws, ws_bytes   unused (may be NULL / 0)
+ * One launch: the blocks of each group are scored by one thread-block cluster
+ * whose CTAs then select the top K_b together. */
 TLS_API tls_status tls_block_score_topk(const tls_shape *s, const void *q, const void *meta, const int32_t *seq_lens,
                                 int32_t *block_idx_out, float *block_score_out, void *ws, size_t ws_bytes,
                                 void *stream);
@@ -150,7 +153,10 @@ TLS_API tls_status tls_block_score_topk(const tls_shape *s, const void *q, const
  *   block_idx       device int32 [B][H_kv][k_b] (ids < 0 are skipped)
  *   token_idx_out   device int32 [B][H_kv][k_t], ascending token positions, -1 padded
  *   token_score_out device fp32 [B][H_kv][k_b * bs] in candidate order, or NULL;
- *                   invalid candidates hold -inf */
+ *                   invalid candidates hold -inf
+ *   ws, ws_bytes    unused (may be NULL / 0)
+ * One launch: the candidates of each group are scored by one thread-block
+ * cluster whose CTAs then select the top K_t together. */
 TLS_API tls_status tls_token_score_topk(const tls_shape *s, const void *q, const void *slab, const int32_t *label_idx,
                                 const int32_t *block_idx, const int32_t *seq_lens, int32_t *token_idx_out,
                                 float *token_score_out, void *ws, size_t ws_bytes, void *stream);
@@ -213,20 +219,18 @@ TLS_API tls_status tls_prefetch_diff(const tls_shape *s, int32_t n_slots, const 
 
 /* Stages 1+2 for callers that cannot allocate device memory (no counterpart in
  * the paper: an addition of this library).  Computes exactly what
- * tls_block_score_topk computes with block_score_out = NULL, but keeps the fp32
- * block scores in a fixed 4 MiB array inside the library's own device memory
- * instead of a caller workspace, so a caller that may not call cudaMalloc and
- * has no spare device buffer (e.g. code running inside another runtime's
- * launch hook) needs only the inputs and block_idx_out.
+ * tls_block_score_topk computes, needs only the inputs and block_idx_out, and
+ * writes the fp32 block scores into a fixed 4 MiB array inside the library's
+ * own device memory instead of a caller buffer (e.g. for code running inside
+ * another runtime's launch hook, which may not call cudaMalloc).
  *   Limit: batch * n_kv_heads * ceil(max_ctx / block_size) <= 1048576 block
  *   scores; larger shapes return TLS_ERR_UNSUPPORTED with a message.
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
  *   before any stream capture.  The array exists on every GPU that loads the
  *   library until the process exits.  All calls on a device share it and it
- *   keeps the last call's scores (each call writes every score it reads, so
- *   nothing needs clearing): calls whose kernels overlap on the GPU race.
- *   Allocates nothing. */
+ *   keeps the last call's scores: calls whose kernels overlap on the GPU
+ *   overwrite each other's scores.  Allocates nothing. */
 TLS_API tls_status tls_block_score_topk_noalloc(const tls_shape *s, const void *q, const void *meta,
                                                 const int32_t *seq_lens, int32_t *block_idx_out, void *stream);
 

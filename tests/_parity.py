@@ -224,10 +224,12 @@ def check_attention(gout: np.ndarray, glse: np.ndarray, oout: np.ndarray, olse: 
     return float(err.max()) if err.size else 0.0
 
 
-def full_stage_parity(w: W.Workload, seq_lens=None, out_dtype=0, name=None):
-    """Every stage against the oracle on one seeded input; returns a summary dict."""
+def full_stage_parity(w: W.Workload, seq_lens=None, out_dtype=0, name=None, inp=None):
+    """Every stage against the oracle on one seeded input (or the given one);
+    returns a summary dict."""
     name = name or w.name
-    inp = W.make_decode_inputs(w, seq_lens=seq_lens)
+    if inp is None:
+        inp = W.make_decode_inputs(w, seq_lens=seq_lens)
     orc = OracleRun(w, inp)
     gpu = GpuInputs(w, inp, out_dtype=out_dtype)
     check_meta(w, inp, gpu, orc)

@@ -67,6 +67,34 @@ def test_full_selection_equals_full_attention_gpu():
     P().full_stage_parity(w, name="full_selection")
 
 
+def periodic_keys(w, period_blocks, seq_lens=None):
+    """Seeded inputs whose keys repeat every `period_blocks` blocks: block
+    summaries, block scores and label-channel token scores then repeat exactly,
+    so both top-k boundaries fall inside long runs of equal scores and the
+    lower-id rule decides which of them are kept."""
+    inp = W.make_decode_inputs(w, seq_lens=seq_lens)
+    P_tok = period_blocks * w.block_size
+    t = np.arange(w.ctx) % P_tok
+    inp.K = np.ascontiguousarray(inp.K[:, :, t])
+    return inp
+
+
+TIES = {
+    # 26 copies of the top block score for k_b = 24; each token score 24 times for k_t = 300
+    "ties_bf16": (W.WORKLOADS["gqa48k_bf16"].with_(batch=2, ctx=4096, k_b=24, k_t=300), 5, [4096, 3999]),
+    "ties_f32_ragged": (W.WORKLOADS["tiny_gqa4k_f32"].with_(batch=3, ctx=1000, k_b=8, k_t=100), 3, [1000, 777, 33]),
+    # the token boundary cuts a run at the largest candidate count (16384)
+    "ties_bf16_kmax": (W.WORKLOADS["gqa48k_bf16"].with_(batch=1, ctx=32768, k_b=512, k_t=5000), 7, None),
+}
+
+
+@pytest.mark.parametrize("name", sorted(TIES))
+def test_tie_heavy_selection_parity(name):
+    w, period, sl = TIES[name]
+    inp = periodic_keys(w, period, seq_lens=sl)
+    P().full_stage_parity(w, name=name, inp=inp)
+
+
 FULL = ["tiny_gqa4k_f32", "gqa48k_bf16", "gqa96k_b8_bf16", "mla64k_b4_bf16"]
 
 

@@ -120,20 +120,19 @@ tls::AttnArgs attn_args(const tls_shape *s) {
   return a;
 }
 
-// Workspace layout: [block scores | attention partials | error word], 256-byte aligned.
+// Workspace layout (attention only), 256-byte aligned regions:
+//   [attention partials][error word]
 struct WsLayout {
-  size_t scores_off, scores_bytes, part_off, part_bytes, err_off, total;
+  size_t part_off, part_bytes, err_off, total;
 };
 
 bool ws_layout(const tls_shape *s, bool paged, WsLayout *w) {
   auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-  w->scores_off = 0;
-  w->scores_bytes = up(static_cast<size_t>(s->batch) * s->n_kv_heads * n_blocks_max(s) * sizeof(float));
   tls::AttnArgs a = attn_args(s);
   a.paged = paged;
   tls::AttnPlan p;
   if (!tls::attn_plan(a, &p)) return false;
-  w->part_off = w->scores_bytes;
+  w->part_off = 0;
   w->part_bytes = up(p.part_floats * sizeof(float));
   w->err_off = w->part_off + w->part_bytes;
   w->total = w->err_off + 256;
@@ -203,28 +202,16 @@ tls_status tls_block_score_topk(const tls_shape *s, const void *q, const void *m
   CHECK_PTR(seq_lens, 4);
   CHECK_PTR(block_idx_out, 4);
   if (block_score_out && !aligned(block_score_out, 4)) return fail(TLS_ERR_INVALID_ARG, "block_score_out misaligned");
-  float *scores = block_score_out;
-  if (!scores) {
-    WsLayout w;
-    if (!ws_layout(s, false, &w)) return fail(TLS_ERR_UNSUPPORTED, "no plan for this shape");
-    if (!ws || ws_bytes < w.scores_off + w.scores_bytes || !aligned(ws, 256))
-      return fail(TLS_ERR_WORKSPACE, "workspace too small or not 256-byte aligned (need %zu bytes)",
-                  w.scores_off + w.scores_bytes);
-    scores = reinterpret_cast<float *>(static_cast<char *>(ws) + w.scores_off);
-  }
-  tls::BlockScoreArgs a{q, meta, seq_lens, scores, block_idx_out, s->batch, s->n_q_heads, s->n_kv_heads, s->d_qk,
-                        s->block_size, n_blocks_max(s), s->max_ctx, s->k_b, s->kv_dtype, device_sms()};
-  cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  st = cuda_status(tls::launch_block_score(a, cs), "block_score launch");
-  if (st != TLS_OK) return st;
-  return cuda_status(tls::launch_block_topk(a, cs), "block_topk launch");
+  (void)ws;  // the selection keeps its keys in on-chip memory: no workspace
+  (void)ws_bytes;
+  tls::BlockScoreArgs a{q, meta, seq_lens, block_score_out, block_idx_out, s->batch, s->n_q_heads, s->n_kv_heads,
+                        s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->k_b, s->kv_dtype};
+  return cuda_status(tls::launch_block_select(a, static_cast<cudaStream_t>(stream)), "block_select launch");
 }
 
 tls_status tls_token_score_topk(const tls_shape *s, const void *q, const void *slab, const int32_t *label_idx,
                                 const int32_t *block_idx, const int32_t *seq_lens, int32_t *token_idx_out,
                                 float *token_score_out, void *ws, size_t ws_bytes, void *stream) {
-  (void)ws;
-  (void)ws_bytes;
   tls_status st = check_shape(s);
   if (st != TLS_OK) return st;
   if (s->batch == 0) return TLS_OK;
@@ -238,7 +225,9 @@ tls_status tls_token_score_topk(const tls_shape *s, const void *q, const void *s
   tls::TokenArgs a{q, slab, label_idx, block_idx, seq_lens, token_idx_out, token_score_out, s->batch, s->n_q_heads,
                    s->n_kv_heads, s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->n_label, s->k_b, s->k_t,
                    s->kv_dtype};
-  return cuda_status(tls::launch_token_topk(a, static_cast<cudaStream_t>(stream)), "token_topk launch");
+  (void)ws;  // the selection keeps its keys in on-chip memory: no workspace
+  (void)ws_bytes;
+  return cuda_status(tls::launch_token_select(a, static_cast<cudaStream_t>(stream)), "token_select launch");
 }
 
 static tls_status attn_common(const tls_shape *s, const void *q, const void *K, const void *V,

@@ -204,171 +204,248 @@ __device__ __forceinline__ int block_excl_scan(int v, int *sh, int &total) {
   return base + incl - v;
 }
 
-// ---------------------------------------------------------------- top-k select
+// ---------------------------------------------------------------- thread-block clusters
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Split cluster barrier: every thread of every CTA of the cluster arrives once
+// and waits once; arrive.release / wait.acquire order the shared-memory stores
+// made before the arrive (local or remote) before the reads after the wait.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_sync() {
+  cluster_arrive();
+  cluster_wait();
+}
+// Shared-memory address of the same variable in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t local_smem_addr, uint32_t rank) {
+  uint32_t a;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local_smem_addr), "r"(rank));
+  return a;
+}
+__device__ __forceinline__ void st_cluster(uint32_t cluster_smem_addr, int v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_smem_addr), "r"(v) : "memory");
+}
+
+// ---------------------------------------------------------------- cluster top-k
 //
-// Selection of the k largest keys among keys[0..n) held in shared memory
-// (key 0 = invalid, never selected; requires 1 <= k <= number of keys > 0),
-// ties to the lower index, output ids ascending.  Steps:
-//   1. histogram of the top 11 key bits (2048 bins), usually fused into the
-//      pass that produces the keys (hist_add);
-//   2. the bin b1 holding the k-th largest key, by a block scan over the bins
-//      taken from the top;
-//   3. the keys of bin b1 are gathered into a short list;
-//   4. two more radix passes (11 then 10 bits) over that list only give the
-//      exact k-th key thr and how many keys equal to thr are kept;
-//   5. an index-ordered compaction: warp w owns a contiguous run of indices
-//      (lane-striped, conflict-free), ranks come from ballots and one block
-//      scan over the warp totals.
+// Selection of the k largest of a group's keys (key 0 = invalid, never
+// selected), ties to the lower index, output ids ascending.  The keys are
+// spread over the CS CTAs of one thread-block cluster: CTA r holds the r-th
+// contiguous slice of the index space in its own shared memory.  Steps:
+//   1. each CTA builds a 256-bin histogram of the top key byte over its slice
+//      while it produces the keys (hist_add);
+//   2. four radix passes of 8 bits (bits 31..24, 23..16, 15..8, 7..0): every
+//      CTA pushes its histogram into an inbox slot of every CTA of the cluster
+//      (distributed shared memory stores), one cluster barrier, and every CTA
+//      sums the CS histograms and finds the same digit of the k-th largest
+//      key; the next pass histograms only the keys that share the digits found
+//      so far.  After pass 4 the k-th key thr is exact, and take_eq says how
+//      many keys equal to thr are kept (the lowest-indexed ones);
+//   3. an index-ordered compaction: inside a CTA, warp w owns a contiguous run
+//      of indices read lane-striped; one pass records ballot masks (lane j
+//      keeps those of steps j, j+32, ...), a block scan of packed
+//      (equal << 16 | greater) counts ranks the steps, the CTA pushes its
+//      packed total to every CTA, one cluster barrier, and the sum over lower
+//      ranks is the CTA's offset; a second pass writes the ids.
+// All cross-CTA traffic is pushed before a cluster barrier and read locally
+// after it, so no CTA touches another's shared memory after the last barrier.
+constexpr int kCBins = 256;
+
+template <int CS>
+struct ClusterSelectSmem {
+  int hist[kCBins];          // this CTA's histogram of the current digit
+  int inbox[2][CS][kCBins];  // histograms pushed by the cluster's CTAs, by pass parity
+  int counts[CS];            // packed (equal << 16 | greater) totals pushed by each CTA
+  int sh[33];
+  int bc[4];
+};
+
+// Adds one valid key's top byte to the histogram.
+__device__ __forceinline__ void hist_add(int *hist, uint32_t key, bool valid) {
+  if (valid) atomicAdd(&hist[key >> 24], 1);
+}
+
 struct SelectResult {
   uint32_t thr;  // the k-th largest key
   int take_eq;   // how many keys equal to thr are kept (the lowest-indexed ones)
 };
 
-constexpr int kHistBins = 2048;
-
-struct SelectSmem {
-  int hist[kHistBins];
-  int sh[33];
-  int bc[4];
-};
-
-// Adds one key's top-11-bit digit to the histogram (`valid` false contributes
-// nothing).  Plain shared-memory atomics: 11-bit digits of score keys are
-// spread, so lanes rarely collide on one bin.
-__device__ __forceinline__ void hist_add(int *hist, uint32_t key, bool valid) {
-  if (valid) atomicAdd(&hist[key >> 21], 1);
-}
-
-template <int NT>
-__device__ __forceinline__ void hist_clear(int *hist) {
-  for (int i = threadIdx.x; i < kHistBins; i += NT) hist[i] = 0;
-}
-
-// Over bins [0, nbins): the bin holding the krem-th largest element, and the
-// number of elements in higher bins.  Thread t owns nbins/NT consecutive bins
-// counted from the top.  Result in bc[0] (bin), bc[1] (count above).
-template <int NT>
-__device__ __forceinline__ void find_bin_from_top(const int *hist, int nbins, int krem, SelectSmem &S) {
-  const int per = nbins / NT;  // nbins is a multiple of NT
-  const int top = nbins - threadIdx.x * per;  // owns bins [top - per, top)
-  int sum = 0;
-  for (int i = 1; i <= per; ++i) sum += hist[top - i];
-  int tot;
-  const int above = block_excl_scan<NT>(sum, S.sh, tot);
-  if (above < krem && krem <= above + sum) {
-    int acc = above;
-    for (int i = 1; i <= per; ++i) {
-      const int c = hist[top - i];
-      if (acc + c >= krem) {
-        S.bc[0] = top - i;
-        S.bc[1] = acc;
-        break;
-      }
-      acc += c;
-    }
-  }
-  __syncthreads();
-}
-
-// Steps 2-4.  hist must hold the step-1 histogram of keys[0..n).  list needs n
-// entries of shared memory.  Contains __syncthreads(); call uniformly.
-template <int NT>
-__device__ SelectResult select_kth(const uint32_t *keys, int n, int k, uint32_t *list, SelectSmem &S) {
-  static_assert(kHistBins % NT == 0 || NT > kHistBins, "bins split evenly over threads");
-  __syncthreads();  // histogram complete
-  find_bin_from_top<NT>(S.hist, kHistBins, k, S);
-  const uint32_t b1 = static_cast<uint32_t>(S.bc[0]);
-  int krem = k - S.bc[1];
-  // gather the keys of bin b1
-  if (threadIdx.x == 0) S.bc[2] = 0;
-  __syncthreads();
-  const int lane = threadIdx.x & 31;
-  for (int base = 0; base < n; base += NT) {
-    const int i = base + threadIdx.x;
-    const uint32_t key = i < n ? keys[i] : 0u;
-    const bool in = i < n && key != 0u && (key >> 21) == b1;
-    const unsigned mask = __ballot_sync(0xffffffffu, in);
-    int slot = 0;
-    if (lane == 0 && mask) slot = atomicAdd(&S.bc[2], __popc(mask));
-    slot = __shfl_sync(0xffffffffu, slot, 0);
-    if (in) list[slot + __popc(mask & ((1u << lane) - 1u))] = key;
-  }
-  __syncthreads();
-  const int m = S.bc[2];
-  // bits 20..10 over the list
-  hist_clear<NT>(S.hist);
-  __syncthreads();
-  for (int i = threadIdx.x; i < m; i += NT) atomicAdd(&S.hist[(list[i] >> 10) & 2047u], 1);
-  __syncthreads();
-  find_bin_from_top<NT>(S.hist, kHistBins, krem, S);
-  const uint32_t b2 = static_cast<uint32_t>(S.bc[0]);
-  krem -= S.bc[1];
-  // bits 9..0 over the list entries of bin b2
-  hist_clear<NT>(S.hist);
-  __syncthreads();
-  for (int i = threadIdx.x; i < m; i += NT) {
-    const uint32_t key = list[i];
-    if (((key >> 10) & 2047u) == b2) atomicAdd(&S.hist[key & 1023u], 1);
-  }
-  __syncthreads();
-  find_bin_from_top<NT>(S.hist, 1024 < NT ? NT : 1024, krem, S);
-  const uint32_t b3 = static_cast<uint32_t>(S.bc[0]);
-  krem -= S.bc[1];
-  return {(b1 << 21) | (b2 << 10) | b3, krem};
-}
-
-// Step 5: ids of the kept keys (key > thr, or key == thr among the first
-// take_eq such keys in index order) in ascending index order to out[0..k), -1
-// to out[k..cap).  id_of(i) maps a key position to the id written.  Warp w owns
-// the contiguous index run [w*seg, (w+1)*seg), read lane-striped; ranks come
-// from ballots and two block scans over the warp totals.
-template <int NT, typename IdOf>
-__device__ void ordered_compact(const uint32_t *keys, int n, SelectResult r, int k, int32_t *out, int cap,
-                                IdOf id_of, SelectSmem &S) {
+// Step 3 inside one CTA.  keys[0..n), n <= CAP.  cta_base(total) receives the
+// CTA's packed (equal << 16 | greater) total and returns the packed total of
+// all lower-indexed keys of the group held elsewhere (0 for a lone CTA).
+// Writes out[p] = id_of(i) for the kept keys at their group-wide ranks p < k.
+template <int NT, int CAP, typename IdOf, typename BaseFn>
+__device__ void ordered_compact(const uint32_t *keys, int n, SelectResult r, int k, int32_t *out, IdOf id_of,
+                                int *sh, BaseFn cta_base) {
   constexpr int NW = NT / 32;
+  constexpr int R = (CAP + NW * 1024 - 1) / (NW * 1024);  // mask slots per lane
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int seg = ((n + NW - 1) / NW + 31) & ~31;  // indices per warp, a multiple of 32
+  const int iters = min(seg >> 5, 32 * R);         // seg >> 5 <= 32 * R when n <= CAP
   const int i0 = wid * seg, i1 = min(i0 + seg, n);
-  const unsigned lt = (1u << lane) - 1u;
-  int n_gt = 0, n_eq = 0;
-#pragma unroll 1
-  for (int base = i0; base < i0 + seg; base += 32) {
-    const int i = base + lane;
+  unsigned gt[R], eq[R];
+#pragma unroll
+  for (int s = 0; s < R; ++s) gt[s] = eq[s] = 0u;
+#pragma unroll 4
+  for (int it = 0; it < iters; ++it) {
+    const int i = i0 + it * 32 + lane;
     const uint32_t key = i < i1 ? keys[i] : 0u;
-    n_gt += __popc(__ballot_sync(0xffffffffu, key > r.thr));
-    n_eq += __popc(__ballot_sync(0xffffffffu, i < i1 && key == r.thr));
+    const unsigned g = __ballot_sync(0xffffffffu, key > r.thr);
+    const unsigned e = __ballot_sync(0xffffffffu, i < i1 && key == r.thr);
+    if ((it & 31) == lane) {
+#pragma unroll
+      for (int s = 0; s < R; ++s)
+        if ((it >> 5) == s) {
+          gt[s] = g;
+          eq[s] = e;
+        }
+    }
   }
-  int tot;
-  const int eq_base = __shfl_sync(0xffffffffu, block_excl_scan<NT>(lane == 0 ? n_eq : 0, S.sh, tot), 0);
-  const int eq_kept = max(0, min(n_eq, r.take_eq - eq_base));
-  int pos = __shfl_sync(0xffffffffu, block_excl_scan<NT>(lane == 0 ? (n_gt + eq_kept) : 0, S.sh, tot), 0);
-  int eq_seen = eq_base;
-#pragma unroll 1
-  for (int base = i0; base < i0 + seg; base += 32) {
-    const int i = base + lane;
-    const uint32_t key = i < i1 ? keys[i] : 0u;
-    const unsigned gtm = __ballot_sync(0xffffffffu, key > r.thr);
-    const unsigned eqm = __ballot_sync(0xffffffffu, i < i1 && key == r.thr);
-    // equal keys of this run that are still within take_eq (lowest lanes first)
-    const int room = max(0, r.take_eq - eq_seen);
-    unsigned keep_eq = eqm;
-    if (__popc(eqm) > room) {
-      keep_eq = 0;
-      unsigned rest = eqm;
+  int pre[R];
+  int run = 0;
+#pragma unroll
+  for (int s = 0; s < R; ++s) {
+    const int pc = (__popc(eq[s]) << 16) | __popc(gt[s]);
+    const int incl = warp_incl_scan(pc);
+    pre[s] = run + incl - pc;
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  int total;
+  const int wexcl = __shfl_sync(0xffffffffu, block_excl_scan<NT>(lane == 0 ? run : 0, sh, total), 0);
+  const int wbase = wexcl + cta_base(total);
+  unsigned sel[R];
+  int pos[R];
+#pragma unroll
+  for (int s = 0; s < R; ++s) {
+    const int before = wbase + pre[s];
+    const int gt_before = before & 0xffff, eq_before = before >> 16;
+    const int room = r.take_eq - eq_before;  // equal keys still to keep at this step
+    unsigned keep = eq[s];
+    if (__popc(keep) > room) {
+      keep = 0u;
+      unsigned rest = eq[s];
       for (int c = 0; c < room; ++c) {
-        keep_eq |= rest & (~rest + 1u);  // lowest set bit
+        keep |= rest & (~rest + 1u);  // lowest set bit
         rest &= rest - 1u;
       }
     }
-    eq_seen += __popc(eqm);
-    const unsigned selm = gtm | keep_eq;
-    if ((selm >> lane) & 1u) {
-      const int p = pos + __popc(selm & lt);
-      if (p < k) out[p] = id_of(i);  // p < k always holds; the guard keeps writes in bounds
-    }
-    pos += __popc(selm);
+    sel[s] = gt[s] | keep;
+    pos[s] = gt_before + min(r.take_eq, eq_before);
   }
-  for (int i = k + threadIdx.x; i < cap; i += NT) out[i] = -1;
+  const unsigned lt = (1u << lane) - 1u;
+#pragma unroll 4
+  for (int it = 0; it < iters; ++it) {
+    unsigned vs = sel[0];
+    int vp = pos[0];
+#pragma unroll
+    for (int s = 1; s < R; ++s)
+      if ((it >> 5) == s) {
+        vs = sel[s];
+        vp = pos[s];
+      }
+    const unsigned selm = __shfl_sync(0xffffffffu, vs, it & 31);
+    const int p0 = __shfl_sync(0xffffffffu, vp, it & 31);
+    if ((selm >> lane) & 1u) {
+      const int p = p0 + __popc(selm & lt);
+      if (p < k) out[p] = id_of(i0 + it * 32 + lane);  // p < k always holds; the guard keeps writes in bounds
+    }
+  }
+}
+
+// The whole selection for one cluster (steps 2-3; step 1 done by the caller
+// into S.hist).  keys[0..n): this CTA's slice, n <= CAP; k_req: wanted count
+// (clamped to the number of valid keys of the group); out[0..cap): ids in
+// ascending order, -1 padded (cap >= k_req).  Every thread of every CTA of the
+// cluster calls it once, after cluster_arrive_relaxed() at kernel entry.
+template <int NT, int CS, int CAP, typename IdOf>
+__device__ void cluster_topk(const uint32_t *keys, int n, int k_req, int32_t *out, int cap, IdOf id_of,
+                             ClusterSelectSmem<CS> &S) {
+  static_assert(NT >= kCBins && NT % 32 == 0, "one histogram bin per thread");
+  const int tid = threadIdx.x;
+  const uint32_t rank = cluster_ctarank();
+  __syncthreads();  // this CTA's keys and histogram are complete
+  cluster_wait();   // every CTA of the cluster has started (entry arrive)
+  uint32_t prefix = 0;
+  int krem = k_req, k = 0;
+#pragma unroll 1
+  for (int p = 0; p < 4; ++p) {
+    const int shift = 24 - 8 * p;
+    if (tid < kCBins) {  // push; the bin is cleared for the next digit by its owner
+      const int v = S.hist[tid];
+      S.hist[tid] = 0;
+      const uint32_t la = smem_addr(&S.inbox[p & 1][rank][tid]);
+#pragma unroll
+      for (int c = 0; c < CS; ++c) st_cluster(cluster_map(la, c), v);
+    }
+    cluster_sync();
+    if (tid < 32) {  // warp 0: lane l owns bins 255-8l .. 248-8l, from the top
+      int cnt[8], sum = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int bin = kCBins - 1 - 8 * tid - i;
+        int v = 0;
+#pragma unroll
+        for (int c = 0; c < CS; ++c) v += S.inbox[p & 1][c][bin];
+        cnt[i] = v;
+        sum += v;
+      }
+      const int incl = warp_incl_scan(sum);
+      if (p == 0) krem = min(k_req, __shfl_sync(0xffffffffu, incl, 31));  // valid keys of the group
+      int acc = incl - sum;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (acc < krem && acc + cnt[i] >= krem) {  // exactly one (lane, bin) satisfies this
+          S.bc[0] = kCBins - 1 - 8 * tid - i;
+          S.bc[1] = acc;
+        }
+        acc += cnt[i];
+      }
+      if (p == 0 && tid == 0) S.bc[2] = krem;
+    }
+    __syncthreads();
+    if (p == 0) {
+      k = S.bc[2];
+      krem = k;
+      if (k <= 0) break;  // the group has no valid key: same decision in every CTA
+    }
+    const uint32_t digit = static_cast<uint32_t>(S.bc[0]);
+    krem -= S.bc[1];
+    prefix |= digit << shift;
+    if (p < 3) {  // next digit over this CTA's keys that share the digits found so far
+      const uint32_t want = prefix >> shift;
+      const int nshift = shift - 8;
+      constexpr int U = 8;
+      for (int base = 0; base < n; base += NT * U) {
+        uint32_t kv[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int i = base + u * NT + tid;
+          kv[u] = i < n ? keys[i] : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u)
+          if (kv[u] != 0u && (kv[u] >> shift) == want) atomicAdd(&S.hist[(kv[u] >> nshift) & 255u], 1);
+      }
+      __syncthreads();
+    }
+  }
+  if (k > 0) {
+    ordered_compact<NT, CAP>(keys, n, SelectResult{prefix, krem}, k, out, id_of, S.sh, [&](int total) {
+      if (tid < CS) st_cluster(cluster_map(smem_addr(&S.counts[rank]), tid), total);
+      cluster_sync();
+      int base = 0;
+      for (uint32_t c = 0; c < rank; ++c) base += S.counts[c];
+      return base;
+    });
+  }
+  if (rank == 0)
+    for (int i = max(k, 0) + tid; i < cap; i += NT) out[i] = -1;
 }
 
 }  // namespace tls

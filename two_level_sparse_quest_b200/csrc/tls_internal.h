@@ -12,26 +12,41 @@ namespace tls {
 // Launch with programmatic dependent launch enabled: the kernel's launch and
 // its pre-wait prologue overlap the tail of the previous kernel in the stream
 // (the kernel itself waits for that grid before touching global memory).
+// cluster_x > 1 also groups the CTAs into thread-block clusters of
+// (cluster_x, 1, 1); grid.x must be a multiple of it.
 template <typename... KArgs, typename... Args>
-inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                              Args &&...args) {
+inline cudaError_t launch_pdl_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                                      int cluster_x, Args &&...args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (cluster_x > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(cluster_x);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args &&...args) {
+  return launch_pdl_cluster(kernel, grid, block, smem, st, 1, static_cast<Args &&>(args)...);
 }
 
 // Records a printf-style message for tls_last_error() on this thread; returns st.
 tls_status set_error(tls_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
 
-constexpr int kMaxSelectKeys = 16384;  // keys held in shared memory by one selection CTA
+constexpr int kMaxSelectKeys = 16384;  // keys of one selection (blocks or candidates of a group)
 
 struct MetaArgs {
   const void *K;
@@ -48,14 +63,12 @@ struct BlockScoreArgs {
   const void *q;
   const void *meta;
   const int32_t *seq_lens;
-  float *scores;      // [B*H_kv][n_blocks_max]
+  float *scores;      // [B*H_kv][n_blocks_max] or null (not written)
   int32_t *block_idx; // [B*H_kv][k_b]
   int batch, n_q_heads, n_kv_heads, d, block_size, n_blocks_max, max_ctx, k_b, dtype;
-  int num_sms;
-  int *err;  // optional: set to 1 when a bounded wait gave up
 };
-cudaError_t launch_block_score(const BlockScoreArgs &a, cudaStream_t st);
-cudaError_t launch_block_topk(const BlockScoreArgs &a, cudaStream_t st);
+// Block score and top-K_b in one launch (one thread-block cluster per group).
+cudaError_t launch_block_select(const BlockScoreArgs &a, cudaStream_t st);
 
 struct TokenArgs {
   const void *q;
@@ -67,7 +80,8 @@ struct TokenArgs {
   float *token_score;  // nullable
   int batch, n_q_heads, n_kv_heads, d, block_size, n_blocks_max, max_ctx, n_label, k_b, k_t, dtype;
 };
-cudaError_t launch_token_topk(const TokenArgs &a, cudaStream_t st);
+// Token score and top-K_t in one launch (one thread-block cluster per group).
+cudaError_t launch_token_select(const TokenArgs &a, cudaStream_t st);
 
 struct AttnArgs {
   const void *q;

@@ -1,24 +1,21 @@
 // tls_noalloc.cu -- block selection for callers that cannot allocate device memory.
 //
-// tls_block_score_topk needs a place for the fp32 block scores between its two
-// kernels (the score pass and the top-K_b pass): either the caller's
-// block_score_out or the caller's workspace.  Some callers have neither and
-// cannot make one: code that runs inside another runtime's launch hook (an
-// inference-engine plugin, a serving loop that forbids device allocation once
-// it is running), where cudaMalloc is not allowed or would synchronise the
-// device in the middle of a step.  tls_block_score_topk_noalloc serves them: it
-// keeps the scores in a fixed array that lives in the library's own device
-// memory (g_noalloc_scores below) and needs no buffer besides the inputs and
-// the block_idx output.  Nothing here allocates.
+// tls_block_score_topk_noalloc serves code that runs inside another runtime's
+// launch hook (an inference-engine plugin, a serving loop that forbids device
+// allocation once it is running), where cudaMalloc is not allowed or would
+// synchronise the device in the middle of a step: it needs no buffer besides
+// the inputs and the block_idx output, and it leaves the step's fp32 block
+// scores in a fixed array that lives in the library's own device memory
+// (g_noalloc_scores below).  The selection itself keeps its keys on chip, so
+// the array only receives the scores; nothing here allocates.
 //
 // The array is 4 MiB (kNoAllocMaxScores fp32 scores) and exists on every GPU
 // that loads the library, until the process exits.  It holds
 // batch * n_kv_heads * ceil(max_ctx / block_size) scores at most; larger shapes
-// are rejected.  Every call writes the scores of all blocks it later reads, so
-// nothing in the array has to start at zero; the array keeps the last call's
-// scores.  All calls on one device share the array: calls whose kernels
-// overlap on the GPU (two streams, or two threads) overwrite each other's
-// scores and race.
+// are rejected.  Every call writes the scores of all its blocks, so nothing in
+// the array has to start at zero; the array keeps the last call's scores.  All
+// calls on one device share the array: calls whose kernels overlap on the GPU
+// (two streams, or two threads) overwrite each other's scores.
 #include <cuda_runtime.h>
 
 #include <cstdio>
