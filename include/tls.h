@@ -234,6 +234,16 @@ TLS_API tls_status tls_prefetch_diff(const tls_shape *s, int32_t n_slots, const 
 TLS_API tls_status tls_block_score_topk_noalloc(const tls_shape *s, const void *q, const void *meta,
                                                 const int32_t *seq_lens, int32_t *block_idx_out, void *stream);
 
+/* Device-side failure flags of the current device.  Kernels that wait on
+ * other CTAs or on the tensor-core/copy engines bound every wait; when one
+ * gives up (which a correct run never sees) the kernel still ends, its outputs
+ * are undefined, and it sets a bit in a library-owned device word:
+ *   1 = an attention kernel's wait, 2 = a selection cluster's exchange wait.
+ * Writes the word to *flags_out (0 = no failure since the last clear) and,
+ * when clear != 0, zeroes it.  Reads with a synchronous cudaMemcpy, so call it
+ * after the work to check has completed. */
+TLS_API tls_status tls_device_error(int32_t *flags_out, int32_t clear);
+
 /* Bounded host wait on a cudaEvent_t: polls until the event completes or
  * timeout_ms elapses.  Returns TLS_OK, TLS_ERR_TIMEOUT, or TLS_ERR_CUDA when
  * the event reports an error.  Never blocks longer than timeout_ms (+ 1 ms). */

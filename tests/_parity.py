@@ -279,6 +279,7 @@ def full_stage_parity(w: W.Workload, seq_lens=None, out_dtype=0, name=None, inp=
                 same_groups += 1
                 hs = slice(g * G, (g + 1) * G)
                 check_attention(cout[b, hs], clse[b, hs], orc.out[b, hs], orc.lse[b, hs], f"{name} chained b{b} g{g}")
+    assert tls().tls_device_error(clear=True) == 0, f"{name}: a kernel's bounded wait gave up"
     res = dict(block_swaps=swaps_b, token_swaps=swaps_t, attn_max_abs_err=err,
                chained_groups_identical=same_groups, groups=w.batch * w.n_kv_heads)
     report(name, **res)

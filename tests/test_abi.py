@@ -116,6 +116,11 @@ def test_pointer_checks(T):
     assert st == T.TLS_ERR_WORKSPACE
 
 
+def test_device_error_checks_its_argument(T):
+    assert T._lib.tls_device_error(None, 0) == T.TLS_ERR_INVALID_ARG
+    assert "flags_out is NULL" in T.tls_last_error()
+
+
 def test_empty_batch_is_a_noop(T):
     s = good_shape(T, batch=0)
     assert T._lib.tls_block_score_topk(ctypes.byref(s), None, None, None, None, None, None, 0, None) == T.TLS_OK

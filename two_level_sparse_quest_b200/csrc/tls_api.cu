@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <chrono>
+#include <mutex>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -120,10 +121,9 @@ tls::AttnArgs attn_args(const tls_shape *s) {
   return a;
 }
 
-// Workspace layout (attention only), 256-byte aligned regions:
-//   [attention partials][error word]
+// Workspace layout (attention only): the split-KV partials, 256-byte aligned.
 struct WsLayout {
-  size_t part_off, part_bytes, err_off, total;
+  size_t part_off, part_bytes, total;
 };
 
 bool ws_layout(const tls_shape *s, bool paged, WsLayout *w) {
@@ -134,12 +134,33 @@ bool ws_layout(const tls_shape *s, bool paged, WsLayout *w) {
   if (!tls::attn_plan(a, &p)) return false;
   w->part_off = 0;
   w->part_bytes = up(p.part_floats * sizeof(float));
-  w->err_off = w->part_off + w->part_bytes;
-  w->total = w->err_off + 256;
+  w->total = w->part_off + w->part_bytes;
   return true;
 }
 
+// The library's device error word: one int per GPU, zero until a kernel's
+// bounded wait gives up (bits kErrAttnWait, kErrSelectWait).
+__device__ int g_device_error;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_err_mu;
+int *g_err_word[kMaxDevices] = {};
+
 }  // namespace
+
+namespace tls {
+int *device_error_word() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_err_mu);
+  if (!g_err_word[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    g_err_word[dev] = static_cast<int *>(p);
+  }
+  return g_err_word[dev];
+}
+}  // namespace tls
 
 namespace tls {
 tls_status set_error(tls_status st, const char *fmt, ...) {
@@ -205,7 +226,8 @@ tls_status tls_block_score_topk(const tls_shape *s, const void *q, const void *m
   (void)ws;  // the selection keeps its keys in on-chip memory: no workspace
   (void)ws_bytes;
   tls::BlockScoreArgs a{q, meta, seq_lens, block_score_out, block_idx_out, s->batch, s->n_q_heads, s->n_kv_heads,
-                        s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->k_b, s->kv_dtype};
+                        s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->k_b, s->kv_dtype,
+                        tls::device_error_word()};
   return cuda_status(tls::launch_block_select(a, static_cast<cudaStream_t>(stream)), "block_select launch");
 }
 
@@ -224,7 +246,7 @@ tls_status tls_token_score_topk(const tls_shape *s, const void *q, const void *s
   if (token_score_out && !aligned(token_score_out, 4)) return fail(TLS_ERR_INVALID_ARG, "token_score_out misaligned");
   tls::TokenArgs a{q, slab, label_idx, block_idx, seq_lens, token_idx_out, token_score_out, s->batch, s->n_q_heads,
                    s->n_kv_heads, s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->n_label, s->k_b, s->k_t,
-                   s->kv_dtype};
+                   s->kv_dtype, tls::device_error_word()};
   (void)ws;  // the selection keeps its keys in on-chip memory: no workspace
   (void)ws_bytes;
   return cuda_status(tls::launch_token_select(a, static_cast<cudaStream_t>(stream)), "token_select launch");
@@ -261,7 +283,7 @@ static tls_status attn_common(const tls_shape *s, const void *q, const void *K, 
   a.out = out;
   a.lse = lse_out;
   a.part = reinterpret_cast<float *>(static_cast<char *>(ws) + w.part_off);
-  a.err = reinterpret_cast<int *>(static_cast<char *>(ws) + w.err_off);
+  a.err = tls::device_error_word();
   a.paged = paged;
   tls::AttnPlan p;
   if (!tls::attn_plan(a, &p)) return fail(TLS_ERR_UNSUPPORTED, "no attention plan for this shape");
@@ -359,6 +381,18 @@ tls_status tls_wait_event(void *event, int32_t timeout_ms) {
     if (ms >= timeout_ms) return fail(TLS_ERR_TIMEOUT, "event not complete after %d ms", timeout_ms);
     std::this_thread::sleep_for(std::chrono::microseconds(200));
   }
+}
+
+tls_status tls_device_error(int32_t *flags_out, int32_t clear) {
+  if (!flags_out) return fail(TLS_ERR_INVALID_ARG, "flags_out is NULL");
+  int *w = tls::device_error_word();
+  if (!w) return fail(TLS_ERR_CUDA, "the device error word could not be looked up on the current device");
+  int v = 0;
+  tls_status st = cuda_status(cudaMemcpy(&v, w, sizeof v, cudaMemcpyDeviceToHost), "reading the device error word");
+  if (st != TLS_OK) return st;
+  *flags_out = v;
+  if (clear && v) return cuda_status(cudaMemset(w, 0, sizeof v), "clearing the device error word");
+  return TLS_OK;
 }
 
 }  // extern "C"

@@ -280,10 +280,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnArgs a, Attn
     const size_t units = static_cast<size_t>(a.batch) * a.n_kv_heads;
     float *ml = a.part + (static_cast<size_t>(unit) * p.max_pieces + piece) * G * 2;
     float *po = a.part + units * p.max_pieces * G * 2 + (static_cast<size_t>(unit) * p.max_pieces + piece) * G * kTcD;
-    if (tid < G) {
-      ml[tid * 2] = m[tid];
-      ml[tid * 2 + 1] = red[tid] + red[8 + tid] + red[16 + tid] + red[24 + tid];
-    }
+#pragma unroll
+    for (int h = 0; h < G; ++h)
+      if (tid == h) {  // m[] indexed by a compile-time h stays in registers
+        ml[h * 2] = m[h];
+        ml[h * 2 + 1] = red[h] + red[8 + h] + red[16 + h] + red[24 + h];
+      }
 #pragma unroll
     for (int h = 0; h < G; ++h) po[h * kTcD + tid] = ov[h] + ov[8 + h];
     __syncthreads();
@@ -411,7 +413,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(AttnArgs a, Attn
   if (cur_unit >= 0 && !failed) flush(cur_unit);
   if (!failed) wait_o();
   cp_async_wait<0>();
-  if (failed && tid == 0) atomicExch(a.err, 1);
+  if (failed && tid == 0 && a.err) atomicOr(a.err, kErrAttnWait);
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {

@@ -211,26 +211,57 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
   return r;
 }
 // Split cluster barrier: every thread of every CTA of the cluster arrives once
-// and waits once; arrive.release / wait.acquire order the shared-memory stores
-// made before the arrive (local or remote) before the reads after the wait.
+// and waits once.
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
-__device__ __forceinline__ void cluster_sync() {
-  cluster_arrive();
-  cluster_wait();
-}
 // Shared-memory address of the same variable in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t cluster_map(uint32_t local_smem_addr, uint32_t rank) {
   uint32_t a;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(a) : "r"(local_smem_addr), "r"(rank));
   return a;
 }
-__device__ __forceinline__ void st_cluster(uint32_t cluster_smem_addr, int v) {
-  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(cluster_smem_addr), "r"(v) : "memory");
+// Asynchronous store into (possibly another CTA's) shared memory that counts
+// its bytes on that CTA's mbarrier (complete_tx).
+__device__ __forceinline__ void st_async_v4(uint32_t cluster_addr, uint4 v, uint32_t cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   cluster_addr),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(cluster_bar)
+               : "memory");
 }
+__device__ __forceinline__ void st_async_b32(uint32_t cluster_addr, uint32_t v, uint32_t cluster_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(cluster_addr), "r"(v),
+               "r"(cluster_bar)
+               : "memory");
+}
+__device__ __forceinline__ void mbarrier_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes) : "memory");
+}
+// Bounded wait (cluster-scope acquire: the awaited bytes were written by other
+// CTAs); false when it gave up after about a second.
+__device__ __forceinline__ bool mbarrier_wait_cluster(uint64_t *bar, uint32_t parity) {
+  for (uint32_t i = 0; i < (1u << 24); ++i) {
+    uint32_t ok;
+    asm volatile(
+        "{\n"
+        " .reg .pred p;\n"
+        " mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n"
+        "}\n"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if (i > 32) __nanosleep(32);
+  }
+  return false;
+}
+
+// Bits of the library's device error word (set by kernels whose bounded wait
+// gave up; read by tls_device_error).
+constexpr int kErrAttnWait = 1;
+constexpr int kErrSelectWait = 2;
 
 // ---------------------------------------------------------------- cluster top-k
 //
@@ -240,31 +271,52 @@ __device__ __forceinline__ void st_cluster(uint32_t cluster_smem_addr, int v) {
 // contiguous slice of the index space in its own shared memory.  Steps:
 //   1. each CTA builds a 256-bin histogram of the top key byte over its slice
 //      while it produces the keys (hist_add);
-//   2. four radix passes of 8 bits (bits 31..24, 23..16, 15..8, 7..0): every
-//      CTA pushes its histogram into an inbox slot of every CTA of the cluster
-//      (distributed shared memory stores), one cluster barrier, and every CTA
-//      sums the CS histograms and finds the same digit of the k-th largest
-//      key; the next pass histograms only the keys that share the digits found
-//      so far.  After pass 4 the k-th key thr is exact, and take_eq says how
-//      many keys equal to thr are kept (the lowest-indexed ones);
+//   2. four radix passes of 8 bits (bits 31..24, 23..16, 15..8, 7..0): warp 0
+//      of every CTA packs its histogram as 16-bit counts and sends it with
+//      asynchronous stores into a per-pass inbox of every CTA of the cluster,
+//      counting the bytes on that CTA's per-pass mbarrier; once its own
+//      mbarrier has all CS histograms, warp 0 sums them and finds the digit of
+//      the k-th largest key (every CTA finds the same one); the next pass
+//      histograms only the keys that share the digits found so far.  After
+//      pass 4 the k-th key thr is exact, and take_eq says how many keys equal
+//      to thr are kept (the lowest-indexed ones);
 //   3. an index-ordered compaction: inside a CTA, warp w owns a contiguous run
 //      of indices read lane-striped; one pass records ballot masks (lane j
 //      keeps those of steps j, j+32, ...), a block scan of packed
-//      (equal << 16 | greater) counts ranks the steps, the CTA pushes its
-//      packed total to every CTA, one cluster barrier, and the sum over lower
+//      (equal << 16 | greater) counts ranks the steps, every CTA sends its
+//      packed total to every CTA (one more mbarrier), and the sum over lower
 //      ranks is the CTA's offset; a second pass writes the ids.
-// All cross-CTA traffic is pushed before a cluster barrier and read locally
-// after it, so no CTA touches another's shared memory after the last barrier.
+// A CTA only waits for bytes addressed to it, so no CTA exits while a store to
+// its shared memory is outstanding; the one cluster barrier (entry arrive,
+// wait before the first send) makes every CTA's mbarriers initialised before
+// anyone sends.  Counts fit 16 bits: a group has at most kSelectCapacity keys.
 constexpr int kCBins = 256;
+constexpr int kSelectCapacity = 16384;
 
 template <int CS>
 struct ClusterSelectSmem {
-  int hist[kCBins];          // this CTA's histogram of the current digit
-  int inbox[2][CS][kCBins];  // histograms pushed by the cluster's CTAs, by pass parity
-  int counts[CS];            // packed (equal << 16 | greater) totals pushed by each CTA
+  int hist[kCBins];           // this CTA's histogram of the current digit
+  uint4 inbox[4][CS][32];     // per pass, per source CTA: lane l's 8 bins (top-down) as 16-bit counts
+  int counts[CS];             // packed (equal << 16 | greater) totals sent by each CTA
+  uint64_t bar[5];            // passes 0..3, counts
   int sh[33];
   int bc[4];
 };
+
+// At kernel entry, before anything else touches S: the mbarriers are armed for
+// the bytes every pass will receive; then the entry cluster arrive.
+template <int CS>
+__device__ __forceinline__ void cluster_topk_begin(ClusterSelectSmem<CS> &S) {
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int i = 0; i < 5; ++i) mbarrier_init(&S.bar[i], 1);
+    mbarrier_init_fence();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mbarrier_arrive_expect_tx(&S.bar[i], CS * 32 * 16);
+    mbarrier_arrive_expect_tx(&S.bar[4], CS * 4);
+  }
+  cluster_arrive_relaxed();
+}
 
 // Adds one valid key's top byte to the histogram.
 __device__ __forceinline__ void hist_add(int *hist, uint32_t key, bool valid) {
@@ -362,38 +414,53 @@ __device__ void ordered_compact(const uint32_t *keys, int n, SelectResult r, int
 // into S.hist).  keys[0..n): this CTA's slice, n <= CAP; k_req: wanted count
 // (clamped to the number of valid keys of the group); out[0..cap): ids in
 // ascending order, -1 padded (cap >= k_req).  Every thread of every CTA of the
-// cluster calls it once, after cluster_arrive_relaxed() at kernel entry.
+// cluster calls it once, after cluster_topk_begin() at kernel entry.  A wait
+// that gives up sets kErrSelectWait in *err (the results are then undefined;
+// the kernel still ends).
 template <int NT, int CS, int CAP, typename IdOf>
 __device__ void cluster_topk(const uint32_t *keys, int n, int k_req, int32_t *out, int cap, IdOf id_of,
-                             ClusterSelectSmem<CS> &S) {
+                             ClusterSelectSmem<CS> &S, int *err) {
   static_assert(NT >= kCBins && NT % 32 == 0, "one histogram bin per thread");
-  const int tid = threadIdx.x;
+  static_assert(CS * CAP <= kSelectCapacity, "16-bit bin counts");
+  const int tid = threadIdx.x, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
   __syncthreads();  // this CTA's keys and histogram are complete
-  cluster_wait();   // every CTA of the cluster has started (entry arrive)
+  cluster_wait();   // every CTA of the cluster has armed its mbarriers
   uint32_t prefix = 0;
   int krem = k_req, k = 0;
+  bool ok = true;
 #pragma unroll 1
   for (int p = 0; p < 4; ++p) {
     const int shift = 24 - 8 * p;
-    if (tid < kCBins) {  // push; the bin is cleared for the next digit by its owner
-      const int v = S.hist[tid];
-      S.hist[tid] = 0;
-      const uint32_t la = smem_addr(&S.inbox[p & 1][rank][tid]);
-#pragma unroll
-      for (int c = 0; c < CS; ++c) st_cluster(cluster_map(la, c), v);
-    }
-    cluster_sync();
     if (tid < 32) {  // warp 0: lane l owns bins 255-8l .. 248-8l, from the top
+      const int top = kCBins - 1 - 8 * lane;
+      uint32_t w[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        w[j] = static_cast<uint32_t>(S.hist[top - 2 * j]) | (static_cast<uint32_t>(S.hist[top - 2 * j - 1]) << 16);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) S.hist[top - j] = 0;  // cleared for the next digit
+      const uint32_t la = smem_addr(&S.inbox[p][rank][lane]);
+      const uint32_t lb = smem_addr(&S.bar[p]);
+      const uint4 v = make_uint4(w[0], w[1], w[2], w[3]);
+#pragma unroll
+      for (int c = 0; c < CS; ++c) st_async_v4(cluster_map(la, c), v, cluster_map(lb, c));
+      ok = mbarrier_wait_cluster(&S.bar[p], 0) && ok;
+      uint32_t sm[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int c = 0; c < CS; ++c) {
+        const uint4 x = S.inbox[p][c][lane];
+        sm[0] += x.x;
+        sm[1] += x.y;
+        sm[2] += x.z;
+        sm[3] += x.w;
+      }
       int cnt[8], sum = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int bin = kCBins - 1 - 8 * tid - i;
-        int v = 0;
-#pragma unroll
-        for (int c = 0; c < CS; ++c) v += S.inbox[p & 1][c][bin];
-        cnt[i] = v;
-        sum += v;
+      for (int j = 0; j < 4; ++j) {
+        cnt[2 * j] = static_cast<int>(sm[j] & 0xffffu);
+        cnt[2 * j + 1] = static_cast<int>(sm[j] >> 16);
+        sum += cnt[2 * j] + cnt[2 * j + 1];
       }
       const int incl = warp_incl_scan(sum);
       if (p == 0) krem = min(k_req, __shfl_sync(0xffffffffu, incl, 31));  // valid keys of the group
@@ -401,12 +468,12 @@ __device__ void cluster_topk(const uint32_t *keys, int n, int k_req, int32_t *ou
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         if (acc < krem && acc + cnt[i] >= krem) {  // exactly one (lane, bin) satisfies this
-          S.bc[0] = kCBins - 1 - 8 * tid - i;
+          S.bc[0] = top - i;
           S.bc[1] = acc;
         }
         acc += cnt[i];
       }
-      if (p == 0 && tid == 0) S.bc[2] = krem;
+      if (p == 0 && lane == 0) S.bc[2] = krem;
     }
     __syncthreads();
     if (p == 0) {
@@ -437,8 +504,10 @@ __device__ void cluster_topk(const uint32_t *keys, int n, int k_req, int32_t *ou
   }
   if (k > 0) {
     ordered_compact<NT, CAP>(keys, n, SelectResult{prefix, krem}, k, out, id_of, S.sh, [&](int total) {
-      if (tid < CS) st_cluster(cluster_map(smem_addr(&S.counts[rank]), tid), total);
-      cluster_sync();
+      if (tid < CS)
+        st_async_b32(cluster_map(smem_addr(&S.counts[rank]), tid), static_cast<uint32_t>(total),
+                     cluster_map(smem_addr(&S.bar[4]), tid));
+      ok = mbarrier_wait_cluster(&S.bar[4], 0) && ok;
       int base = 0;
       for (uint32_t c = 0; c < rank; ++c) base += S.counts[c];
       return base;
@@ -446,6 +515,7 @@ __device__ void cluster_topk(const uint32_t *keys, int n, int k_req, int32_t *ou
   }
   if (rank == 0)
     for (int i = max(k, 0) + tid; i < cap; i += NT) out[i] = -1;
+  if (!ok && err) atomicOr(err, kErrSelectWait);
 }
 
 }  // namespace tls

@@ -43,6 +43,10 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return launch_pdl_cluster(kernel, grid, block, smem, st, 1, static_cast<Args &&>(args)...);
 }
 
+// Device address of the library's error word on the current device (null if
+// it cannot be looked up): kernels whose bounded wait gives up set a bit in it.
+int *device_error_word();
+
 // Records a printf-style message for tls_last_error() on this thread; returns st.
 tls_status set_error(tls_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
 
@@ -66,6 +70,7 @@ struct BlockScoreArgs {
   float *scores;      // [B*H_kv][n_blocks_max] or null (not written)
   int32_t *block_idx; // [B*H_kv][k_b]
   int batch, n_q_heads, n_kv_heads, d, block_size, n_blocks_max, max_ctx, k_b, dtype;
+  int *err;           // the library's device error word
 };
 // Block score and top-K_b in one launch (one thread-block cluster per group).
 cudaError_t launch_block_select(const BlockScoreArgs &a, cudaStream_t st);
@@ -79,6 +84,7 @@ struct TokenArgs {
   int32_t *token_idx;
   float *token_score;  // nullable
   int batch, n_q_heads, n_kv_heads, d, block_size, n_blocks_max, max_ctx, n_label, k_b, k_t, dtype;
+  int *err;           // the library's device error word
 };
 // Token score and top-K_t in one launch (one thread-block cluster per group).
 cudaError_t launch_token_select(const TokenArgs &a, cudaStream_t st);
@@ -93,7 +99,7 @@ struct AttnArgs {
   void *out;
   float *lse;
   float *part;  // workspace partials
-  int *err;     // workspace word: set to 1 when a bounded wait in a kernel gave up
+  int *err;     // the library's device error word (kErrAttnWait when a bounded wait gave up)
   int batch, n_q_heads, n_kv_heads, d_qk, d_v, v_is_k_prefix, block_size, n_blocks_max, max_ctx, k_t;
   int dtype, out_dtype, paged;
   float scale_log2;  // softmax_scale * log2(e)

@@ -14,8 +14,9 @@
 // chunks (coalesced, non-allocating loads), the row sum is a segmented warp
 // reduction.  The scores become order-preserving keys in the CTA's shared
 // memory and the cluster selects the top K_b (cluster_topk: 8-bit radix
-// passes over histograms exchanged through distributed shared memory, then an
-// index-ordered compaction; ties to the lower block id).
+// passes over histograms exchanged between the CTAs with asynchronous
+// distributed-shared-memory stores, then an index-ordered compaction; ties to
+// the lower block id).
 // Stage 3+4 (token score and top-K_t, (de) section 2.A "Stufe 2", (es) section
 // 2.A.2): CTA r scores the r-th slice of the group's K_b * bs candidates from
 // the label-channel slab (a block's rows are contiguous) against
@@ -48,7 +49,7 @@ __global__ void __launch_bounds__(kScoreThreads, NCH > 32 ? 2 : 4) block_select_
   constexpr int U = CPL >= 4 ? 2 : 4;                 // rows in flight per warp (per lane: U * CPL loads)
   extern __shared__ float qpm[];                      // [2d]: Q^+ then Q^-, then the slice's keys
   __shared__ ClusterSelectSmem<CS> S;
-  cluster_arrive_relaxed();
+  cluster_topk_begin(S);
   const int group = blockIdx.y;
   const int b = group / a.n_kv_heads, g = group % a.n_kv_heads;
   const int G = a.n_q_heads / a.n_kv_heads;
@@ -134,7 +135,7 @@ __global__ void __launch_bounds__(kScoreThreads, NCH > 32 ? 2 : 4) block_select_
   }
   cluster_topk<kScoreThreads, CS, kSliceCap>(
       keys, max(r1 - r0, 0), a.k_b, a.block_idx + static_cast<size_t>(group) * a.k_b, a.k_b,
-      [r0](int i) { return r0 + i; }, S);
+      [r0](int i) { return r0 + i; }, S, a.err);
 }
 
 // RCH: 16-byte chunks per slab row (r * bytes / 16), 1..8.  grid = (CS, groups),
@@ -149,7 +150,7 @@ __global__ void __launch_bounds__(kTokThreads, RCH > 2 ? 2 : 4) token_select_ker
   __shared__ int blk[1024];           // block ids of the slice's blocks
   __shared__ float qbar[64];
   __shared__ ClusterSelectSmem<CS> S;
-  cluster_arrive_relaxed();
+  cluster_topk_begin(S);
   const int group = blockIdx.y;
   const int b = group / a.n_kv_heads, g = group % a.n_kv_heads;
   const int G = a.n_q_heads / a.n_kv_heads;
@@ -228,7 +229,7 @@ __global__ void __launch_bounds__(kTokThreads, RCH > 2 ? 2 : 4) token_select_ker
         const int jb = blk_of(j);
         return blk[jb - jb0] * bs + (j - jb * bs);
       },
-      S);
+      S, a.err);
 }
 
 template <typename E, int NCH>

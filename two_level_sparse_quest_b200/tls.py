@@ -30,7 +30,7 @@ STATUS_NAMES = {0: "TLS_OK", 1: "TLS_ERR_INVALID_ARG", 2: "TLS_ERR_UNSUPPORTED",
 
 EXPORTED = ("tls_version", "tls_last_error", "tls_workspace_size", "tls_build_block_meta", "tls_block_score_topk",
             "tls_token_score_topk", "tls_sparse_attn_decode", "tls_sparse_attn_decode_paged", "tls_offload_reset",
-            "tls_prefetch_diff", "tls_wait_event", "tls_block_score_topk_noalloc")
+            "tls_prefetch_diff", "tls_wait_event", "tls_block_score_topk_noalloc", "tls_device_error")
 
 
 class TlsShape(ctypes.Structure):
@@ -65,6 +65,7 @@ _sigs = {
     "tls_prefetch_diff": ([_S, _i32, _P, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "tls_wait_event": ([_P, _i32], ctypes.c_int),
     "tls_block_score_topk_noalloc": ([_S, _P, _P, _P, _P, _P], ctypes.c_int),
+    "tls_device_error": ([ctypes.POINTER(_i32), _i32], ctypes.c_int),
 }
 for _name, (_args, _ret) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -199,3 +200,11 @@ def tls_wait_event(event, timeout_ms: int) -> int:
     if st not in (TLS_OK, TLS_ERR_TIMEOUT):
         _check(st, "tls_wait_event")
     return st
+
+
+def tls_device_error(clear: bool = False) -> int:
+    """Failure flags of the current device (1: an attention wait gave up,
+    2: a selection exchange wait gave up); 0 means none since the last clear."""
+    v = _i32(0)
+    _check(_lib.tls_device_error(ctypes.byref(v), int(bool(clear))), "tls_device_error")
+    return v.value
