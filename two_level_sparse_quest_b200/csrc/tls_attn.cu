@@ -366,7 +366,7 @@ struct Variant {
   int warps, head_chunk;
 };
 
-constexpr int kStages = 3;
+constexpr int kStages = 2;
 
 template <typename E, int D, int DV, int HG, bool VPREFIX>
 constexpr int warps_of() {
@@ -413,26 +413,34 @@ cudaError_t dispatch_gqa(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) 
 
 }  // namespace
 
-// GQA bf16 d = 128 has two kernels: the CUDA-core one (default; faster on the
-// 96k decode workload, where the gather is the bound) and the tcgen05 one
-// (TLS_ATTN_IMPL=tensor_core; read once per process).
-static bool tensor_core_allowed() {
-  static int allowed = -1;
-  if (allowed < 0) {
+// Kernel choice.  bf16 GQA shapes run the warp-MMA kernel (tls_attn_mma.cu)
+// by default; TLS_ATTN_IMPL=cuda_core selects this file's CUDA-core kernel and
+// TLS_ATTN_IMPL=tensor_core the tcgen05 kernel (bf16, d = 128) instead.  The
+// variable is read once per process.  Other shapes (fp32, latent attention)
+// always run the CUDA-core kernel.
+enum ImplChoice { kImplDefault = 0, kImplCudaCore = 1, kImplTcgen05 = 2 };
+static int impl_choice() {
+  static int choice = -1;
+  if (choice < 0) {
     const char *e = getenv("TLS_ATTN_IMPL");
-    allowed = (e && strcmp(e, "tensor_core") == 0) ? 1 : 0;
+    if (e && strcmp(e, "tensor_core") == 0) choice = kImplTcgen05;
+    else if (e && strcmp(e, "cuda_core") == 0) choice = kImplCudaCore;
+    else choice = kImplDefault;
   }
-  return allowed == 1;
+  return choice;
 }
 
 bool attn_plan(const AttnArgs &a, AttnPlan *p) {
-  if (tensor_core_allowed() && attn_tc_supported(a)) {
-    p->tensor_core = 1;
+  const int choice = impl_choice();
+  if (choice == kImplTcgen05 && attn_tc_supported(a)) {
+    p->impl = 1;
     return attn_tc_plan(a, p);
   }
-  p->tensor_core = 0;
+  const bool mma = choice == kImplDefault && attn_mma_supported(a);
+  p->impl = mma ? 2 : 0;
   Variant v;
   if (!pick_variant(a, &v)) return false;
+  if (mma) v.warps = attn_mma_warps(a);
   const int G = a.n_q_heads / a.n_kv_heads;
   p->warps_per_cta = v.warps;
   p->tokens_per_tile = kTT;
@@ -453,7 +461,8 @@ bool attn_plan(const AttnArgs &a, AttnPlan *p) {
 }
 
 static cudaError_t launch_split(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) {
-  if (p.tensor_core) return launch_attention_tc(a, p, st);
+  if (p.impl == 1) return launch_attention_tc(a, p, st);
+  if (p.impl == 2) return launch_attention_mma(a, p, st);
   if (a.v_is_k_prefix) return run_attention<BF16, 576, 512, 4, true, false, kStages>(a, p, st);
   if (a.dtype == 1) {
     if (a.d_qk == 128) return a.paged ? dispatch_gqa<BF16, 128, true>(a, p, st) : dispatch_gqa<BF16, 128, false>(a, p, st);
