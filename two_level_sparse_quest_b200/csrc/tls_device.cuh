@@ -97,11 +97,6 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem, bool pr
   int n = pred ? 16 : 0;  // 0 source bytes -> the 16 bytes are zero-filled
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(s), "l"(gmem), "r"(n) : "memory");
 }
-// 4-byte asynchronous copy (an index), completing with the thread's cp.async groups.
-__device__ __forceinline__ void cp_async4(void *smem, const void *gmem) {
-  unsigned s = static_cast<unsigned>(__cvta_generic_to_shared(smem));
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(s), "l"(gmem) : "memory");
-}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
