@@ -57,6 +57,8 @@ def algorithmic_bytes(w) -> dict:
     # per stage (what each C call must read/write)
     parts["stage_block"] = parts["block_summary"] + parts["q"] + G * w.k_b * 4
     parts["stage_token"] = parts["label_slab"] + parts["q"] + G * (w.k_b + w.k_t) * 4
+    # stages 1-4 in one launch (tls_select_step): the block ids go out and come back once
+    parts["stage_select"] = parts["stage_block"] + parts["stage_token"] - parts["q"]
     parts["stage_attn"] = parts["gathered_kv"] + parts["q"] + parts["out_lse"] + G * w.k_t * 4
     return parts
 
@@ -226,18 +228,15 @@ def gpu_arm(args, rank, world, local_rank):
     def step(L, ev=None):
         if ev:
             ev[0].record(stream)
-        T.tls_block_score_topk(shape, L.q, L.meta, seq_lens, bidx, None, ws, sh)
+        T.tls_select_step(shape, L.q, L.meta, L.slab, label, seq_lens, bidx, tidx, None, None, sh)
         if ev:
             ev[1].record(stream)
-        T.tls_token_score_topk(shape, L.q, L.slab, label, bidx, seq_lens, tidx, None, ws, sh)
-        if ev:
-            ev[2].record(stream)
         T.tls_sparse_attn_decode(shape, L.q, L.K, L.V, tidx, out, lse, ws, sh)
         if ev:
-            ev[3].record(stream)
+            ev[2].record(stream)
 
-    # block score with its top-k tail, token score with its top-k tail, attention split, merge
-    launches_per_step = 4
+    # stages 1-4 (one cluster launch), attention split, log-sum-exp merge
+    launches_per_step = 3
     for i in range(args.warmup):
         step(layers[i % N_LAYERS])
     torch.cuda.synchronize()
@@ -246,7 +245,7 @@ def gpu_arm(args, rank, world, local_rank):
     # programmatic dependent launch; per-stage CUDA events (which break that
     # overlap at the stage boundaries) are recorded on every SAMPLE-th step only.
     SAMPLE = 8
-    evs = {i: [torch.cuda.Event(enable_timing=True) for _ in range(4)] for i in range(0, args.steps, SAMPLE)}
+    evs = {i: [torch.cuda.Event(enable_timing=True) for _ in range(3)] for i in range(0, args.steps, SAMPLE)}
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
@@ -267,7 +266,7 @@ def gpu_arm(args, rank, world, local_rank):
         dist.barrier()
     clocks = sampler.stop() if rank == 0 else None
     ms = t_start.elapsed_time(t_end)
-    st = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3])] for e in evs.values()])
+    st = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2])] for e in evs.values()])
     stage_ms = st.mean(axis=0)
     ms = max_over_ranks(ms, dev)
 
@@ -308,7 +307,7 @@ def gpu_arm(args, rank, world, local_rank):
     ab = algorithmic_bytes(w)
     peaks = read_peaks()
     step_ms = ms / args.steps
-    names = ["stage_block", "stage_token", "stage_attn"]
+    names = ["stage_select", "stage_attn"]
     dom = int(np.argmax(stage_ms))
     dom_bytes = ab[names[dom]]
     achieved = dom_bytes / (stage_ms[dom] * 1e-3) / 1e9

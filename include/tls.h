@@ -161,6 +161,17 @@ TLS_API tls_status tls_token_score_topk(const tls_shape *s, const void *q, const
                                 const int32_t *block_idx, const int32_t *seq_lens, int32_t *token_idx_out,
                                 float *token_score_out, void *ws, size_t ws_bytes, void *stream);
 
+/* Stages 1-4 in one launch: exactly what tls_block_score_topk followed by
+ * tls_token_score_topk compute (same arithmetic, same bits), with each
+ * group's thread-block cluster going from its block selection straight to its
+ * token stage instead of waiting for every group's block selection.
+ * Arguments as in those two calls; block_idx_out is written and then read
+ * back by the same launch.  block_score_out / token_score_out may be NULL. */
+TLS_API tls_status tls_select_step(const tls_shape *s, const void *q, const void *meta, const void *slab,
+                                   const int32_t *label_idx, const int32_t *seq_lens, int32_t *block_idx_out,
+                                   int32_t *token_idx_out, float *block_score_out, float *token_score_out,
+                                   void *stream);
+
 /* Stage 5: exact attention over the selected tokens.
  * gist.science (es) section 2.A.2: the final attention over the K_t kept tokens
  * at token precision.  For each query head h:

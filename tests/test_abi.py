@@ -116,6 +116,15 @@ def test_pointer_checks(T):
     assert st == T.TLS_ERR_WORKSPACE
 
 
+def test_select_step_checks_before_launch(T):
+    s = good_shape(T)
+    st = T._lib.tls_select_step(ctypes.byref(s), 256, 256, None, 256, 256, 256, 256, None, None, None)
+    assert st == T.TLS_ERR_INVALID_ARG and "slab is NULL" in T.tls_last_error()
+    bad = good_shape(T, k_b=600)
+    st = T._lib.tls_select_step(ctypes.byref(bad), 256, 256, 256, 256, 256, 256, 256, None, None, None)
+    assert st == T.TLS_ERR_UNSUPPORTED
+
+
 def test_device_error_checks_its_argument(T):
     assert T._lib.tls_device_error(None, 0) == T.TLS_ERR_INVALID_ARG
     assert "flags_out is NULL" in T.tls_last_error()

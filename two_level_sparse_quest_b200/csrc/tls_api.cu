@@ -252,6 +252,30 @@ tls_status tls_token_score_topk(const tls_shape *s, const void *q, const void *s
   return cuda_status(tls::launch_token_select(a, static_cast<cudaStream_t>(stream)), "token_select launch");
 }
 
+tls_status tls_select_step(const tls_shape *s, const void *q, const void *meta, const void *slab,
+                           const int32_t *label_idx, const int32_t *seq_lens, int32_t *block_idx_out,
+                           int32_t *token_idx_out, float *block_score_out, float *token_score_out, void *stream) {
+  tls_status st = check_shape(s);
+  if (st != TLS_OK) return st;
+  if (s->batch == 0) return TLS_OK;
+  CHECK_PTR(q, 16);
+  CHECK_PTR(meta, 16);
+  CHECK_PTR(slab, 16);
+  CHECK_PTR(label_idx, 4);
+  CHECK_PTR(seq_lens, 4);
+  CHECK_PTR(block_idx_out, 4);
+  CHECK_PTR(token_idx_out, 4);
+  if (block_score_out && !aligned(block_score_out, 4)) return fail(TLS_ERR_INVALID_ARG, "block_score_out misaligned");
+  if (token_score_out && !aligned(token_score_out, 4)) return fail(TLS_ERR_INVALID_ARG, "token_score_out misaligned");
+  int *err = tls::device_error_word();
+  tls::BlockScoreArgs a{q, meta, seq_lens, block_score_out, block_idx_out, s->batch, s->n_q_heads, s->n_kv_heads,
+                        s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->k_b, s->kv_dtype, err};
+  tls::TokenArgs t{q, slab, label_idx, block_idx_out, seq_lens, token_idx_out, token_score_out, s->batch, s->n_q_heads,
+                   s->n_kv_heads, s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->n_label, s->k_b, s->k_t,
+                   s->kv_dtype, err};
+  return cuda_status(tls::launch_select_step(a, t, static_cast<cudaStream_t>(stream)), "select_step launch");
+}
+
 static tls_status attn_common(const tls_shape *s, const void *q, const void *K, const void *V,
                               const int32_t *token_idx, const int32_t *slot_of_block, int32_t n_slots, void *out,
                               float *lse_out, void *ws, size_t ws_bytes, void *stream, bool paged) {

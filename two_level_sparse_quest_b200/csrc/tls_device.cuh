@@ -215,6 +215,9 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 // Shared-memory address of the same variable in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t cluster_map(uint32_t local_smem_addr, uint32_t rank) {
@@ -306,7 +309,7 @@ struct ClusterSelectSmem {
 // At kernel entry, before anything else touches S: the mbarriers are armed for
 // the bytes every pass will receive; then the entry cluster arrive.
 template <int CS>
-__device__ __forceinline__ void cluster_topk_begin(ClusterSelectSmem<CS> &S) {
+__device__ __forceinline__ void cluster_topk_arm(ClusterSelectSmem<CS> &S) {
   if (threadIdx.x == 0) {
 #pragma unroll
     for (int i = 0; i < 5; ++i) mbarrier_init(&S.bar[i], 1);
@@ -315,6 +318,10 @@ __device__ __forceinline__ void cluster_topk_begin(ClusterSelectSmem<CS> &S) {
     for (int i = 0; i < 4; ++i) mbarrier_arrive_expect_tx(&S.bar[i], CS * 32 * 16);
     mbarrier_arrive_expect_tx(&S.bar[4], CS * 4);
   }
+}
+template <int CS>
+__device__ __forceinline__ void cluster_topk_begin(ClusterSelectSmem<CS> &S) {
+  cluster_topk_arm(S);
   cluster_arrive_relaxed();
 }
 
@@ -414,18 +421,20 @@ __device__ void ordered_compact(const uint32_t *keys, int n, SelectResult r, int
 // into S.hist).  keys[0..n): this CTA's slice, n <= CAP; k_req: wanted count
 // (clamped to the number of valid keys of the group); out[0..cap): ids in
 // ascending order, -1 padded (cap >= k_req).  Every thread of every CTA of the
-// cluster calls it once, after cluster_topk_begin() at kernel entry.  A wait
+// cluster calls it once per ClusterSelectSmem, after cluster_topk_begin() on
+// that smem at kernel entry; entry_wait = false for a later selection whose
+// mbarriers were armed before an earlier call's entry wait.  A wait
 // that gives up sets kErrSelectWait in *err (the results are then undefined;
 // the kernel still ends).
 template <int NT, int CS, int CAP, typename IdOf>
 __device__ void cluster_topk(const uint32_t *keys, int n, int k_req, int32_t *out, int cap, IdOf id_of,
-                             ClusterSelectSmem<CS> &S, int *err) {
+                             ClusterSelectSmem<CS> &S, int *err, bool entry_wait = true) {
   static_assert(NT >= kCBins && NT % 32 == 0, "one histogram bin per thread");
   static_assert(CS * CAP <= kSelectCapacity, "16-bit bin counts");
   const int tid = threadIdx.x, lane = tid & 31;
   const uint32_t rank = cluster_ctarank();
   __syncthreads();  // this CTA's keys and histogram are complete
-  cluster_wait();   // every CTA of the cluster has armed its mbarriers
+  if (entry_wait) cluster_wait();  // every CTA of the cluster has armed its mbarriers
   uint32_t prefix = 0;
   int krem = k_req, k = 0;
   bool ok = true;

@@ -88,6 +88,8 @@ struct TokenArgs {
 };
 // Token score and top-K_t in one launch (one thread-block cluster per group).
 cudaError_t launch_token_select(const TokenArgs &a, cudaStream_t st);
+// Stages 1-4 in one launch: the group's cluster selects its blocks, then its tokens.
+cudaError_t launch_select_step(const BlockScoreArgs &a, const TokenArgs &t, cudaStream_t st);
 
 struct AttnArgs {
   const void *q;

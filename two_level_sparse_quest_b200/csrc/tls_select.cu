@@ -1,5 +1,5 @@
 // tls_select.cu -- the two selection stages of the AsyncTLS decode step, each
-// one launch of one thread-block cluster per (sequence, KV head) group.
+// run by one thread-block cluster per (sequence, KV head) group.
 //
 // Stage 1+2 (block score and top-K_b, gist.science (de) section 2.A "Stufe 1"
 // + "Optimierung"; (es) section 2.A.1): the Quest-style bound of a block j for
@@ -22,6 +22,11 @@
 // the label-channel slab (a block's rows are contiguous) against
 // Qbar_L = sum_h q_h[L] in fp32, and the cluster selects the top K_t the same
 // way (ties to the lower token position).
+// Three kernels: stages 1+2, stages 3+4, and all four in one launch (the
+// cluster goes from its block selection straight to its token stage; the
+// selected block ids pass through global memory behind a release/acquire
+// cluster barrier).  The arithmetic is shared, so the fused launch gives the
+// same bits as the two separate ones.
 #include <algorithm>
 
 #include "tls_device.cuh"
@@ -32,41 +37,31 @@ namespace {
 
 constexpr int kClusterSize = 8;  // CTAs per group (portable cluster size)
 constexpr int kSliceCap = kMaxSelectKeys / kClusterSize;  // keys per CTA
-constexpr int kScoreThreads = 256;
-constexpr int kTokThreads = 256;
+constexpr int kThreads = 256;
 
-// NCH: 16-byte chunks per summary row (2 * d * bytes / 16).  grid = (CS, groups),
-// cluster = (CS, 1, 1).  The first rows' loads are issued before the head fold
-// so that the query reads overlap them.
-template <typename E, int NCH, int CS>
-__global__ void __launch_bounds__(kScoreThreads, NCH > 32 ? 2 : 4) block_select_kernel(BlockScoreArgs a, int rows_per_cta) {
+// ---------------------------------------------------------------- stage 1 body
+// After the grid dependency wait: folds the group's query into qpm = [Q+; Q-]
+// and scores summary rows [r0, r1) into keys[row - r0] and hist (top key
+// byte).  NCH: 16-byte chunks per summary row (2 * d * bytes / 16).  The first
+// rows' loads are issued before the head fold so that the query reads
+// overlap them.
+template <typename E, int NCH>
+__device__ __forceinline__ void score_blocks(const BlockScoreArgs &a, int group, int nb, int r0, int r1, float *qpm,
+                                             uint32_t *keys, int *hist) {
   constexpr int EPC = E::kEPC;
-  constexpr int LPR = NCH < 32 ? NCH : 32;            // lanes per row
-  constexpr int RPW = 32 / LPR;                       // rows per warp step
-  constexpr int CPL = (NCH + 31) / 32;                // chunks per lane
-  constexpr int NWARP = kScoreThreads / 32;
+  constexpr int LPR = NCH < 32 ? NCH : 32;  // lanes per row
+  constexpr int RPW = 32 / LPR;             // rows per warp step
+  constexpr int CPL = (NCH + 31) / 32;      // chunks per lane
+  constexpr int NWARP = kThreads / 32;
   constexpr int STEP = NWARP * RPW;
-  constexpr int U = CPL >= 4 ? 2 : 4;                 // rows in flight per warp (per lane: U * CPL loads)
-  extern __shared__ float qpm[];                      // [2d]: Q^+ then Q^-, then the slice's keys
-  __shared__ ClusterSelectSmem<CS> S;
-  cluster_topk_begin(S);
-  const int group = blockIdx.y;
+  constexpr int U = CPL >= 4 ? 2 : 4;  // rows in flight per warp (per lane: U * CPL loads)
   const int b = group / a.n_kv_heads, g = group % a.n_kv_heads;
   const int G = a.n_q_heads / a.n_kv_heads;
   const int d = a.d;
-  const int nbm = a.n_blocks_max;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int sub = lane / LPR, cl = lane % LPR;  // row within the warp step, chunk lane
-  const int rank = static_cast<int>(cluster_ctarank());
-  uint32_t *keys = reinterpret_cast<uint32_t *>(qpm + 2 * d);
-  if (threadIdx.x < kCBins) S.hist[threadIdx.x] = 0;
-  grid_dependency_wait();
-  const int sq = min(max(a.seq_lens[b], 0), a.max_ctx);
-  const int nb = (sq + a.block_size - 1) / a.block_size;
-  const int r0 = rank * rows_per_cta;
-  const int r1 = min(r0 + rows_per_cta, nbm);
-  const char *meta = static_cast<const char *>(a.meta) + static_cast<size_t>(group) * nbm * (NCH * 16);
-  float *out = a.scores ? a.scores + static_cast<size_t>(group) * nbm : nullptr;
+  const char *meta = static_cast<const char *>(a.meta) + static_cast<size_t>(group) * a.n_blocks_max * (NCH * 16);
+  float *out = a.scores ? a.scores + static_cast<size_t>(group) * a.n_blocks_max : nullptr;
   auto load_rows = [&](int rb, uint4 (&v)[U][CPL]) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -83,7 +78,7 @@ __global__ void __launch_bounds__(kScoreThreads, NCH > 32 ? 2 : 4) block_select_
   uint4 v[U][CPL];
   int rb = r0 + warp * RPW;
   load_rows(rb, v);  // in flight while the query is folded
-  for (int i = threadIdx.x; i < d; i += kScoreThreads) {
+  for (int i = threadIdx.x; i < d; i += kThreads) {
     float pos = 0.f, neg = 0.f;
     for (int hh = 0; hh < G; ++hh) {
       const float x = load_elem<E>(a.q, (static_cast<size_t>(b) * a.n_q_heads + g * G + hh) * d + i);
@@ -122,7 +117,7 @@ __global__ void __launch_bounds__(kScoreThreads, NCH > 32 ? 2 : 4) block_select_
         const bool valid = row < nb;
         const uint32_t key = valid ? max(score_key(acc), 1u) : 0u;
         keys[row - r0] = key;
-        hist_add(S.hist, key, valid);
+        hist_add(hist, key, valid);
         if (out) out[row] = valid ? acc : -INFINITY;
       }
     }
@@ -133,44 +128,14 @@ __global__ void __launch_bounds__(kScoreThreads, NCH > 32 ? 2 : 4) block_select_
         for (int j = 0; j < CPL; ++j) v[u][j] = nv[u][j];
     }
   }
-  cluster_topk<kScoreThreads, CS, kSliceCap>(
-      keys, max(r1 - r0, 0), a.k_b, a.block_idx + static_cast<size_t>(group) * a.k_b, a.k_b,
-      [r0](int i) { return r0 + i; }, S, a.err);
 }
 
-// RCH: 16-byte chunks per slab row (r * bytes / 16), 1..8.  grid = (CS, groups),
-// cluster = (CS, 1, 1); CTA r scores candidates [r*per, (r+1)*per).
-template <typename E, int RCH, int CS>
-__global__ void __launch_bounds__(kTokThreads, RCH > 2 ? 2 : 4) token_select_kernel(TokenArgs a, int per_cta) {
-  using S_t = typename E::storage;
-  constexpr int EPC = E::kEPC;
-  constexpr int NT = kTokThreads;
-  constexpr int kBatch = RCH <= 4 ? 4 : 2;  // candidates whose rows a thread loads at once
-  extern __shared__ uint32_t keys[];  // [per_cta]
-  __shared__ int blk[1024];           // block ids of the slice's blocks
-  __shared__ float qbar[64];
-  __shared__ ClusterSelectSmem<CS> S;
-  cluster_topk_begin(S);
-  const int group = blockIdx.y;
+// Qbar_L[c] = sum_h q_h[L[c]] (fp32, heads in order) into qbar[0..r).
+template <typename E>
+__device__ __forceinline__ void fold_label_query(const TokenArgs &a, int group, float *qbar) {
   const int b = group / a.n_kv_heads, g = group % a.n_kv_heads;
   const int G = a.n_q_heads / a.n_kv_heads;
-  const int bs = a.block_size, r = a.n_label;
-  const int C = a.k_b * bs;
-  const int rank = static_cast<int>(cluster_ctarank());
-  const int c0 = min(rank * per_cta, C), c1 = min(c0 + per_cta, C);
-  const bool bs_pow2 = (bs & (bs - 1)) == 0;
-  const int bs_shift = __ffs(bs) - 1;
-  auto blk_of = [&](int j) { return bs_pow2 ? (j >> bs_shift) : (j / bs); };
-  const int jb0 = c0 < c1 ? blk_of(c0) : 0;
-  const int nblk = c0 < c1 ? blk_of(c1 - 1) - jb0 + 1 : 0;  // <= min(k_b, 1024)
-  if (threadIdx.x < kCBins) S.hist[threadIdx.x] = 0;
-  grid_dependency_wait();
-  const int seq = min(max(a.seq_lens[b], 0), a.max_ctx);
-  for (int i = threadIdx.x; i < nblk; i += NT) {
-    const int v = a.block_idx[static_cast<size_t>(group) * a.k_b + jb0 + i];
-    blk[i] = (v >= 0 && v < a.n_blocks_max) ? v : -1;
-  }
-  for (int c = threadIdx.x; c < r; c += NT) {
+  for (int c = threadIdx.x; c < a.n_label; c += kThreads) {
     const int ch = a.label_idx[c];
     float sum = 0.f;
     if (ch >= 0 && ch < a.d)
@@ -178,18 +143,34 @@ __global__ void __launch_bounds__(kTokThreads, RCH > 2 ? 2 : 4) token_select_ker
         sum += load_elem<E>(a.q, (static_cast<size_t>(b) * a.n_q_heads + g * G + hh) * a.d + ch);
     qbar[c] = sum;
   }
-  __syncthreads();
+}
+
+// ---------------------------------------------------------------- stage 3 body
+// Scores candidates [c0, c1) of the group (blk[j / bs - jb0] = kept block id,
+// < 0 for none; qbar in shared memory, complete) into keys[j - c0] and hist.
+// RCH: 16-byte chunks per slab row (r * bytes / 16), 1..8.
+template <typename E, int RCH>
+__device__ __forceinline__ void score_tokens(const TokenArgs &a, int group, int seq, int c0, int c1, const int *blk,
+                                             int jb0, const float *qbar, uint32_t *keys, int *hist) {
+  using S_t = typename E::storage;
+  constexpr int EPC = E::kEPC;
+  constexpr int kBatch = RCH <= 4 ? 4 : 2;  // candidates whose rows a thread loads at once
+  const int bs = a.block_size, r = a.n_label;
+  const int C = a.k_b * bs;
+  const bool bs_pow2 = (bs & (bs - 1)) == 0;
+  const int bs_shift = __ffs(bs) - 1;
+  auto blk_of = [&](int j) { return bs_pow2 ? (j >> bs_shift) : (j / bs); };
   float ql[RCH * EPC];
 #pragma unroll
   for (int e = 0; e < RCH * EPC; ++e) ql[e] = qbar[e];  // r == RCH * EPC
   const S_t *slab = static_cast<const S_t *>(a.slab) + static_cast<size_t>(group) * a.max_ctx * r;
   float *score_out = a.token_score ? a.token_score + static_cast<size_t>(group) * C : nullptr;
-  for (int base = c0; base < c1; base += NT * kBatch) {
+  for (int base = c0; base < c1; base += kThreads * kBatch) {
     uint4 v[kBatch][RCH];
     int tok[kBatch];
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
-      const int j = base + u * NT + threadIdx.x;
+      const int j = base + u * kThreads + threadIdx.x;
       int t = -1;
       if (j < c1) {
         const int jb = blk_of(j);
@@ -204,7 +185,7 @@ __global__ void __launch_bounds__(kTokThreads, RCH > 2 ? 2 : 4) token_select_ker
     }
 #pragma unroll
     for (int u = 0; u < kBatch; ++u) {
-      const int j = base + u * NT + threadIdx.x;
+      const int j = base + u * kThreads + threadIdx.x;
       float acc = 0.f;
 #pragma unroll
       for (int c = 0; c < RCH; ++c) {
@@ -219,17 +200,152 @@ __global__ void __launch_bounds__(kTokThreads, RCH > 2 ? 2 : 4) token_select_ker
         keys[j - c0] = key;
         if (score_out) score_out[j] = ok ? acc : -INFINITY;
       }
-      hist_add(S.hist, key, ok);
+      hist_add(hist, key, ok);
     }
   }
-  cluster_topk<NT, CS, kSliceCap>(
-      keys, c1 - c0, a.k_t, a.token_idx + static_cast<size_t>(group) * a.k_t, a.k_t,
+}
+
+// Candidate slice [c0, c1) of cluster rank `rank` and the range of kept-block
+// list entries it covers: [jb0, jb0 + nblk), nblk <= min(k_b, 1024).
+struct TokenSlice {
+  int c0, c1, jb0, nblk;
+};
+__device__ __forceinline__ TokenSlice token_slice(const TokenArgs &a, int rank, int per_cta) {
+  const int bs = a.block_size, C = a.k_b * bs;
+  TokenSlice s;
+  s.c0 = min(rank * per_cta, C);
+  s.c1 = min(s.c0 + per_cta, C);
+  s.jb0 = s.c0 < s.c1 ? s.c0 / bs : 0;
+  s.nblk = s.c0 < s.c1 ? (s.c1 - 1) / bs - s.jb0 + 1 : 0;
+  return s;
+}
+
+// ---------------------------------------------------------------- kernels
+// grid = (CS, groups), cluster = (CS, 1, 1) for all three.
+template <typename E, int NCH, int CS>
+__global__ void __launch_bounds__(kThreads, NCH > 32 ? 2 : 4) block_select_kernel(BlockScoreArgs a, int rows_per_cta) {
+  extern __shared__ float qpm[];  // [2d]: Q^+ then Q^-, then the slice's keys
+  __shared__ ClusterSelectSmem<CS> S;
+  cluster_topk_begin(S);
+  const int group = blockIdx.y;
+  const int rank = static_cast<int>(cluster_ctarank());
+  uint32_t *keys = reinterpret_cast<uint32_t *>(qpm + 2 * a.d);
+  if (threadIdx.x < kCBins) S.hist[threadIdx.x] = 0;
+  grid_dependency_wait();
+  const int b = group / a.n_kv_heads;
+  const int sq = min(max(a.seq_lens[b], 0), a.max_ctx);
+  const int nb = (sq + a.block_size - 1) / a.block_size;
+  const int r0 = rank * rows_per_cta;
+  const int r1 = min(r0 + rows_per_cta, a.n_blocks_max);
+  score_blocks<E, NCH>(a, group, nb, r0, r1, qpm, keys, S.hist);
+  cluster_topk<kThreads, CS, kSliceCap>(
+      keys, max(r1 - r0, 0), a.k_b, a.block_idx + static_cast<size_t>(group) * a.k_b, a.k_b,
+      [r0](int i) { return r0 + i; }, S, a.err);
+}
+
+template <typename E, int RCH, int CS>
+__global__ void __launch_bounds__(kThreads, RCH > 2 ? 2 : 4) token_select_kernel(TokenArgs a, int per_cta) {
+  extern __shared__ uint32_t keys[];  // [per_cta]
+  __shared__ int blk[1024];           // block ids of the slice's blocks
+  __shared__ float qbar[64];
+  __shared__ ClusterSelectSmem<CS> S;
+  cluster_topk_begin(S);
+  const int group = blockIdx.y;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const TokenSlice sl = token_slice(a, rank, per_cta);
+  if (threadIdx.x < kCBins) S.hist[threadIdx.x] = 0;
+  grid_dependency_wait();
+  const int seq = min(max(a.seq_lens[group / a.n_kv_heads], 0), a.max_ctx);
+  for (int i = threadIdx.x; i < sl.nblk; i += kThreads) {
+    const int v = a.block_idx[static_cast<size_t>(group) * a.k_b + sl.jb0 + i];
+    blk[i] = (v >= 0 && v < a.n_blocks_max) ? v : -1;
+  }
+  fold_label_query<E>(a, group, qbar);
+  __syncthreads();
+  score_tokens<E, RCH>(a, group, seq, sl.c0, sl.c1, blk, sl.jb0, qbar, keys, S.hist);
+  const int bs = a.block_size, jb0 = sl.jb0, c0 = sl.c0;
+  cluster_topk<kThreads, CS, kSliceCap>(
+      keys, sl.c1 - sl.c0, a.k_t, a.token_idx + static_cast<size_t>(group) * a.k_t, a.k_t,
       [&](int i) {
         const int j = c0 + i;
-        const int jb = blk_of(j);
+        const int jb = j / bs;
         return blk[jb - jb0] * bs + (j - jb * bs);
       },
       S, a.err);
+}
+
+struct StepArgs {
+  BlockScoreArgs blk;
+  TokenArgs tok;
+};
+
+template <typename E, int NCH, int RCH, int CS>
+__global__ void __launch_bounds__(kThreads, (NCH > 32 || RCH > 2) ? 2 : 4)
+    select_step_kernel(StepArgs s, int rows_per_cta, int per_cta) {
+  extern __shared__ float qpm[];  // [2d] Q^+, Q^-; block keys [rows_per_cta]; token keys [per_cta]
+  __shared__ ClusterSelectSmem<CS> SB, ST;
+  __shared__ int blk[1024];
+  __shared__ float qbar[64];
+  const BlockScoreArgs &a = s.blk;
+  const TokenArgs &t = s.tok;
+  cluster_topk_arm(SB);
+  cluster_topk_arm(ST);
+  cluster_arrive_relaxed();
+  const int group = blockIdx.y;
+  const int rank = static_cast<int>(cluster_ctarank());
+  uint32_t *bkeys = reinterpret_cast<uint32_t *>(qpm + 2 * a.d);
+  uint32_t *tkeys = bkeys + rows_per_cta;
+  if (threadIdx.x < kCBins) {
+    SB.hist[threadIdx.x] = 0;
+    ST.hist[threadIdx.x] = 0;
+  }
+  grid_dependency_wait();
+  const int b = group / a.n_kv_heads;
+  const int sq = min(max(a.seq_lens[b], 0), a.max_ctx);
+  const int nb = (sq + a.block_size - 1) / a.block_size;
+  fold_label_query<E>(t, group, qbar);  // independent of the block stage; complete by the next barrier
+  // ---- stages 1 + 2
+  const int r0 = rank * rows_per_cta;
+  const int r1 = min(r0 + rows_per_cta, a.n_blocks_max);
+  score_blocks<E, NCH>(a, group, nb, r0, r1, qpm, bkeys, SB.hist);
+  int32_t *bout = a.block_idx + static_cast<size_t>(group) * a.k_b;
+  cluster_topk<kThreads, CS, kSliceCap>(
+      bkeys, max(r1 - r0, 0), a.k_b, bout, a.k_b, [r0](int i) { return r0 + i; }, SB, a.err);
+  // every CTA's block ids are in global memory and visible to the cluster
+  cluster_arrive_release();
+  cluster_wait();
+  // ---- stages 3 + 4
+  const TokenSlice sl = token_slice(t, rank, per_cta);
+  for (int i = threadIdx.x; i < sl.nblk; i += kThreads) {
+    const int v = __ldcg(bout + sl.jb0 + i);
+    blk[i] = (v >= 0 && v < t.n_blocks_max) ? v : -1;
+  }
+  __syncthreads();
+  score_tokens<E, RCH>(t, group, sq, sl.c0, sl.c1, blk, sl.jb0, qbar, tkeys, ST.hist);
+  const int bs = t.block_size, jb0 = sl.jb0, c0 = sl.c0;
+  cluster_topk<kThreads, CS, kSliceCap>(
+      tkeys, sl.c1 - sl.c0, t.k_t, t.token_idx + static_cast<size_t>(group) * t.k_t, t.k_t,
+      [&](int i) {
+        const int j = c0 + i;
+        const int jb = j / bs;
+        return blk[jb - jb0] * bs + (j - jb * bs);
+      },
+      ST, t.err, /*entry_wait=*/false);
+}
+
+// ---------------------------------------------------------------- launchers
+// Raises the kernel's dynamic shared-memory limit to `bytes` when a launch
+// needs more than the previous ones on this device (static + dynamic above
+// 48 KB needs the opt-in).  One cache per kernel instantiation (the caller's
+// static array).
+template <typename K>
+cudaError_t allow_smem(K kern, size_t bytes, int (&allowed)[64]) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || allowed[dev] >= static_cast<int>(bytes)) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e == cudaSuccess) allowed[dev] = static_cast<int>(bytes);
+  return e;
 }
 
 template <typename E, int NCH>
@@ -237,18 +353,49 @@ cudaError_t run_block_select(const BlockScoreArgs &a, cudaStream_t st) {
   constexpr int CS = kClusterSize;
   const int rows = (a.n_blocks_max + CS - 1) / CS;  // <= kSliceCap
   const size_t smem = 2 * static_cast<size_t>(a.d) * sizeof(float) + static_cast<size_t>(rows) * sizeof(uint32_t);
-  return launch_pdl_cluster(block_select_kernel<E, NCH, CS>, dim3(CS, a.batch * a.n_kv_heads), dim3(kScoreThreads),
-                            smem, st, CS, a, rows);
+  static int allowed[64] = {};
+  cudaError_t e = allow_smem(block_select_kernel<E, NCH, CS>, smem, allowed);
+  if (e != cudaSuccess) return e;
+  return launch_pdl_cluster(block_select_kernel<E, NCH, CS>, dim3(CS, a.batch * a.n_kv_heads), dim3(kThreads), smem,
+                            st, CS, a, rows);
 }
 
 template <typename E, int RCH>
 cudaError_t run_token_select(const TokenArgs &a, cudaStream_t st) {
   constexpr int CS = kClusterSize;
-  const int C = a.k_b * a.block_size;
-  const int per = (C + CS - 1) / CS;  // <= kSliceCap
+  const int per = (a.k_b * a.block_size + CS - 1) / CS;  // <= kSliceCap
   const size_t smem = static_cast<size_t>(per) * sizeof(uint32_t);
-  return launch_pdl_cluster(token_select_kernel<E, RCH, CS>, dim3(CS, a.batch * a.n_kv_heads), dim3(kTokThreads),
-                            smem, st, CS, a, per);
+  static int allowed[64] = {};
+  cudaError_t e = allow_smem(token_select_kernel<E, RCH, CS>, smem, allowed);
+  if (e != cudaSuccess) return e;
+  return launch_pdl_cluster(token_select_kernel<E, RCH, CS>, dim3(CS, a.batch * a.n_kv_heads), dim3(kThreads), smem,
+                            st, CS, a, per);
+}
+
+template <typename E, int NCH, int RCH>
+cudaError_t run_select_step(const BlockScoreArgs &a, const TokenArgs &t, cudaStream_t st) {
+  constexpr int CS = kClusterSize;
+  const int rows = (a.n_blocks_max + CS - 1) / CS;
+  const int per = (t.k_b * t.block_size + CS - 1) / CS;
+  const size_t smem = 2 * static_cast<size_t>(a.d) * sizeof(float) +
+                      (static_cast<size_t>(rows) + static_cast<size_t>(per)) * sizeof(uint32_t);
+  auto kern = select_step_kernel<E, NCH, RCH, CS>;
+  static int allowed[64] = {};
+  cudaError_t e = allow_smem(kern, smem, allowed);
+  if (e != cudaSuccess) return e;
+  return launch_pdl_cluster(kern, dim3(CS, a.batch * a.n_kv_heads), dim3(kThreads), smem, st, CS, StepArgs{a, t},
+                            rows, per);
+}
+
+template <typename E, int NCH>
+cudaError_t step_by_rch(const BlockScoreArgs &a, const TokenArgs &t, cudaStream_t st) {
+  switch (t.n_label * E::kBytes / 16) {
+    case 1: return run_select_step<E, NCH, 1>(a, t, st);
+    case 2: return run_select_step<E, NCH, 2>(a, t, st);
+    case 4: return run_select_step<E, NCH, 4>(a, t, st);
+    case 8: return run_select_step<E, NCH, 8>(a, t, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
@@ -277,6 +424,23 @@ cudaError_t launch_token_select(const TokenArgs &a, cudaStream_t st) {
     case 2: return a.dtype == 1 ? run_token_select<BF16, 2>(a, st) : run_token_select<F32, 2>(a, st);
     case 4: return a.dtype == 1 ? run_token_select<BF16, 4>(a, st) : run_token_select<F32, 4>(a, st);
     case 8: return a.dtype == 1 ? run_token_select<BF16, 8>(a, st) : run_token_select<F32, 8>(a, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_select_step(const BlockScoreArgs &a, const TokenArgs &t, cudaStream_t st) {
+  const int nch = 2 * a.d * (a.dtype == 1 ? 2 : 4) / 16;
+  if (a.dtype == 1) {
+    switch (nch) {
+      case 16: return step_by_rch<BF16, 16>(a, t, st);
+      case 32: return step_by_rch<BF16, 32>(a, t, st);
+      case 144: return step_by_rch<BF16, 144>(a, t, st);
+    }
+  } else {
+    switch (nch) {
+      case 32: return step_by_rch<F32, 32>(a, t, st);
+      case 64: return step_by_rch<F32, 64>(a, t, st);
+    }
   }
   return cudaErrorInvalidValue;
 }

@@ -30,7 +30,7 @@ STATUS_NAMES = {0: "TLS_OK", 1: "TLS_ERR_INVALID_ARG", 2: "TLS_ERR_UNSUPPORTED",
 
 EXPORTED = ("tls_version", "tls_last_error", "tls_workspace_size", "tls_build_block_meta", "tls_block_score_topk",
             "tls_token_score_topk", "tls_sparse_attn_decode", "tls_sparse_attn_decode_paged", "tls_offload_reset",
-            "tls_prefetch_diff", "tls_wait_event", "tls_block_score_topk_noalloc", "tls_device_error")
+            "tls_prefetch_diff", "tls_wait_event", "tls_block_score_topk_noalloc", "tls_device_error", "tls_select_step")
 
 
 class TlsShape(ctypes.Structure):
@@ -66,6 +66,7 @@ _sigs = {
     "tls_wait_event": ([_P, _i32], ctypes.c_int),
     "tls_block_score_topk_noalloc": ([_S, _P, _P, _P, _P, _P], ctypes.c_int),
     "tls_device_error": ([ctypes.POINTER(_i32), _i32], ctypes.c_int),
+    "tls_select_step": ([_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
 }
 for _name, (_args, _ret) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -157,6 +158,13 @@ def tls_token_score_topk(shape, q, slab, label_idx, block_idx, seq_lens, token_i
     _check(_lib.tls_token_score_topk(ctypes.byref(shape), _ptr(q), _ptr(slab), _ptr(label_idx), _ptr(block_idx),
                                      _ptr(seq_lens), _ptr(token_idx_out), _ptr(token_score_out), wp, wb,
                                      _stream(stream)), "tls_token_score_topk")
+
+
+def tls_select_step(shape, q, meta, slab, label_idx, seq_lens, block_idx_out, token_idx_out, block_score_out=None,
+                    token_score_out=None, stream=None):
+    _check(_lib.tls_select_step(ctypes.byref(shape), _ptr(q), _ptr(meta), _ptr(slab), _ptr(label_idx),
+                                _ptr(seq_lens), _ptr(block_idx_out), _ptr(token_idx_out), _ptr(block_score_out),
+                                _ptr(token_score_out), _stream(stream)), "tls_select_step")
 
 
 def tls_sparse_attn_decode(shape, q, K, V, token_idx, out, lse_out=None, ws=None, stream=None):
