@@ -314,19 +314,20 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(AttnArgs a, AttnPlan p)
                     static_cast<size_t>(unit) * p.max_pieces * HG * DV + hh * DV + ch;
   float M = -INFINITY, Lsum = 0.f, o = 0.f;
   for (int q0 = 0; q0 < n_pieces; q0 += 32) {
-    const int q = q0 + lane;
-    const float mq = q < n_pieces ? ml[(q * HG + hh) * 2] : -INFINITY;
-    const float lq = q < n_pieces ? ml[(q * HG + hh) * 2 + 1] : 0.f;
-    const float Mn = fmaxf(M, warp_max(mq));
-    if (Mn == -INFINITY) continue;
-    const float scale_old = ex2(M - Mn);
-    const float wq = ex2(mq - Mn);
-    Lsum = Lsum * scale_old + warp_sum(wq * lq);
-    o *= scale_old;
+    // all loads of the chunk first (none depends on another): one round trip
     const int nq = min(32, n_pieces - q0);
     float v[32];
 #pragma unroll
     for (int k = 0; k < 32; ++k) v[k] = k < nq ? po[static_cast<size_t>(q0 + k) * HG * DV] : 0.f;
+    const int q = q0 + lane;
+    const float mq = q < n_pieces ? ml[(q * HG + hh) * 2] : -INFINITY;
+    const float lq = q < n_pieces ? ml[(q * HG + hh) * 2 + 1] : 0.f;
+    const float Mn = fmaxf(M, warp_max(mq));
+    const bool any = Mn != -INFINITY;  // false: no token of the unit so far
+    const float scale_old = any ? ex2(M - Mn) : 1.f;
+    const float wq = any ? ex2(mq - Mn) : 0.f;
+    Lsum = Lsum * scale_old + warp_sum(wq * lq);
+    o *= scale_old;
 #pragma unroll
     for (int k = 0; k < 32; ++k) o = fmaf(__shfl_sync(0xffffffffu, wq, k), v[k], o);
     M = Mn;
