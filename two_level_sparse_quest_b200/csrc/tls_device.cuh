@@ -479,6 +479,7 @@ __device__ void cluster_topk(const uint32_t *keys, int n, int k_req, int32_t *ou
         if (acc < krem && acc + cnt[i] >= krem) {  // exactly one (lane, bin) satisfies this
           S.bc[0] = top - i;
           S.bc[1] = acc;
+          S.bc[3] = cnt[i];
         }
         acc += cnt[i];
       }
@@ -493,6 +494,14 @@ __device__ void cluster_topk(const uint32_t *keys, int n, int k_req, int32_t *ou
     const uint32_t digit = static_cast<uint32_t>(S.bc[0]);
     krem -= S.bc[1];
     prefix |= digit << shift;
+    // Exact fit: the bin holds exactly the keys still wanted, so every key at
+    // or above the bin's lowest key is kept and no further digit is needed
+    // (thr = that key - 1, no equal keys taken).  Same decision in every CTA.
+    if (krem == S.bc[3] && prefix != 0u) {
+      prefix -= 1u;
+      krem = 0;
+      break;
+    }
     if (p < 3) {  // next digit over this CTA's keys that share the digits found so far
       const uint32_t want = prefix >> shift;
       const int nshift = shift - 8;
