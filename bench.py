@@ -375,6 +375,105 @@ def gpu_arm(args, rank, world, local_rank):
     return res
 
 
+# ----------------------------------------------------------------------------- offload stream
+def offload_arm(args):
+    """The offload engine on the streaming workload (stream96k_bf16): the full KV
+    lives in pinned host memory, a 2*K_b-slot block cache on the GPU.  One step:
+    block top-K_b from q_t (compute stream); on a copy stream, tls_prefetch_diff
+    loads the blocks of S(t) that are not resident over PCIe while the compute
+    stream scores the tokens of S(t-1) and runs the paged attention (after the
+    copy of step t-1).  The whole query stream is timed with CUDA events; the
+    PCIe bytes per step come from an untimed replay that reads the copy counts."""
+    import numpy as np
+    import torch
+
+    from two_level_sparse_quest_b200 import build as tls_build
+
+    tls_build.build()
+    from two_level_sparse_quest_b200 import tls as T
+    from two_level_sparse_quest_b200 import workloads as W
+
+    dev = torch.device("cuda", 0)
+    w = W.WORKLOADS["stream96k_bf16"]
+    s = T.shape_from_workload(w)
+    inp = W.make_decode_inputs(w)
+    qs = W.make_query_stream(w)
+    steps = qs.shape[0]
+    B, H, nb, bs, d = w.batch, w.n_kv_heads, w.n_blocks, w.block_size, w.d_qk
+    n_slots = 2 * w.k_b
+
+    def up(a):
+        return torch.from_numpy(np.ascontiguousarray(a.view(np.int16) if a.dtype == np.uint16 else a)).to(dev)
+
+    K = up(inp.K)
+    sl, lab = up(inp.seq_lens), up(inp.label_idx)
+    meta = torch.zeros((B, H, nb, 2, d), dtype=torch.int16, device=dev)
+    slab = torch.zeros((B, H, w.ctx, w.n_label), dtype=torch.int16, device=dev)
+    T.tls_build_block_meta(s, K, sl, lab, meta, slab)
+    torch.cuda.synchronize()
+    del K
+    host_kv = torch.from_numpy(W.paged_host_kv(inp).view(np.int16)).pin_memory()
+    cache = torch.zeros((B, H, n_slots, 2, bs, d), dtype=torch.int16, device=dev)
+    sob = torch.empty((B, H, nb), dtype=torch.int32, device=dev)
+    bos = torch.empty((B, H, n_slots), dtype=torch.int32, device=dev)
+    jobs = torch.empty((B, H, w.k_b, 2), dtype=torch.int32, device=dev)
+    n_new = torch.empty((B, H), dtype=torch.int32, device=dev)
+    ws = torch.zeros(T.tls_workspace_size(s), dtype=torch.uint8, device=dev)
+    ring = [torch.empty((B, H, w.k_b), dtype=torch.int32, device=dev) for _ in range(3)]
+    tidx = torch.empty((B, H, w.k_t), dtype=torch.int32, device=dev)
+    out = torch.empty((B, w.n_q_heads, w.d_v), dtype=torch.float32, device=dev)
+    lse = torch.empty((B, w.n_q_heads), dtype=torch.float32, device=dev)
+    q_dev = [up(qs[t]) for t in range(steps)]
+    compute = torch.cuda.current_stream(dev)
+    copy = torch.cuda.Stream(dev)
+    ev_sel = [torch.cuda.Event() for _ in range(2)]
+    ev_copy = [torch.cuda.Event() for _ in range(2)]
+
+    def run(count=False):
+        T.tls_offload_reset(s, n_slots, sob, bos)
+        copied = 0
+        for t in range(steps):
+            cur, prev = ring[t % 3], (ring[(t - 1) % 3] if t else None)
+            T.tls_block_score_topk(s, q_dev[t], meta, sl, cur, None, ws)
+            ev_sel[t % 2].record(compute)
+            copy.wait_event(ev_sel[t % 2])
+            T.tls_prefetch_diff(s, n_slots, host_kv, cache, sob, bos, prev, cur, n_new, jobs, stream=copy)
+            ev_copy[t % 2].record(copy)
+            T.tls_token_score_topk(s, q_dev[t], slab, lab, cur if t == 0 else prev, sl, tidx, None, ws)
+            compute.wait_event(ev_copy[t % 2] if t == 0 else ev_copy[(t - 1) % 2])
+            T.tls_sparse_attn_decode_paged(s, q_dev[t], cache, sob, n_slots, tidx, out, lse, ws)
+            if count:
+                torch.cuda.synchronize()
+                copied += int(n_new.sum())
+        compute.wait_event(ev_copy[(steps - 1) % 2])
+        return copied
+
+    run()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(compute)
+    copy.wait_event(e0)
+    run()
+    e1.record(compute)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    copied = run(count=True)
+    block_bytes = 2 * bs * d * 2
+    return {
+        "metric": "offload decode steps/s (block select, PCIe prefetch of new blocks, paged attention)",
+        "value": steps / (ms * 1e-3), "unit": "steps/s", "n_gpus": 1, "steps": steps,
+        "ms_per_step": ms / steps, "higher_is_better": True, "dtype": "bf16",
+        "data": "synthetic: seeded K/V, AR(1) query stream",
+        "config": {"workload": "stream96k_bf16", "batch": B, "n_q_heads": w.n_q_heads, "n_kv_heads": H,
+                   "d_qk": d, "ctx": w.ctx, "block_size": bs, "k_b": w.k_b, "k_t": w.k_t, "n_slots": n_slots,
+                   "host_kv_bytes": int(host_kv.numel() * 2)},
+        "pcie_bytes_per_step": copied * block_bytes / steps,
+        "pcie_gbs": copied * block_bytes / (ms * 1e-3) / 1e9,
+        "blocks_copied": copied, "first_step_blocks": B * H * w.k_b,
+        "gpu_launches_per_step": 6,
+    }
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_sample(args, budget_s: float):
     """The fp64 oracle (single thread) on a bounded sample of the workload: the
@@ -437,6 +536,8 @@ def main():
     ap.add_argument("--workload", default="gqa96k_b8_bf16")
     ap.add_argument("--impl", default="tls", choices=["tls", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--offload", action="store_true",
+                    help="time the offload engine on the streaming workload instead (one JSON line of its own)")
     ap.add_argument("--layers", type=int, default=N_LAYERS_DEFAULT,
                     help="layer copies rotated through (4 keeps the per-rotation working set above L2)")
     args = ap.parse_args()
@@ -446,6 +547,11 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.offload:
+        if rank == 0:
+            print(json.dumps(offload_arm(args)), flush=True)
+        return
 
     if args.impl == "reference":
         res = reference_arm(args, rank, world)
