@@ -114,10 +114,19 @@ __global__ void __launch_bounds__(MmaLayout<D, NS>::W * 32, 1) attn_mma_kernel(A
   const int Gt = a.n_q_heads / a.n_kv_heads;
 
   // Gather the K and V rows of tile t into stage st (the caller commits).
-  auto issue = [&](int t, int st) {
+  // Issue cursor: tile iss_t (its unit = group, tile within the group, ring
+  // stage) advances by counting, so no integer division sits on the per-tile
+  // path.  A unit is one GQA group (the plan has one head chunk per group).
+  int iss_t = t_begin, iss_group = t_begin / p.tiles_per_group, iss_tile = t_begin % p.tiles_per_group, iss_st = 0;
+  auto issue_next = [&]() {
+    const int t = iss_t, st = iss_st, tile = iss_tile, group = iss_group;
+    if (++iss_tile == p.tiles_per_group) {
+      iss_tile = 0;
+      ++iss_group;
+    }
+    ++iss_t;
+    if (++iss_st == NS) iss_st = 0;
     if (t < t_end) {
-      const int unit = t / p.tiles_per_group, tile = t % p.tiles_per_group;
-      const int group = unit / p.n_head_chunks;
       long long off = -1;
       if (lane < kMT) {
         const int j = tile * kMT + lane;
@@ -182,11 +191,10 @@ __global__ void __launch_bounds__(MmaLayout<D, NS>::W * 32, 1) attn_mma_kernel(A
     }
   };
 
-  auto start_unit = [&](int unit) {
-    const int group = unit / p.n_head_chunks, hc = unit % p.n_head_chunks;
-    const int b = group / a.n_kv_heads, gk = group % a.n_kv_heads;
+  auto start_unit = [&](int unit) {  // unit = group
+    const int b = unit / a.n_kv_heads, gk = unit % a.n_kv_heads;
     const uint32_t *q = static_cast<const uint32_t *>(a.q);
-    const size_t row = (static_cast<size_t>(b) * a.n_q_heads + gk * Gt + hc * HG + g) * D;
+    const size_t row = (static_cast<size_t>(b) * a.n_q_heads + gk * Gt + g) * D;
 #pragma unroll
     for (int kk = 0; kk < KS; ++kk) {
       qa[kk][0] = g < HG ? q[(row + 16 * kk + tq) / 2] : 0u;
@@ -201,17 +209,17 @@ __global__ void __launch_bounds__(MmaLayout<D, NS>::W * 32, 1) attn_mma_kernel(A
   const int mi = lane >> 3, mr = lane & 7;  // ldmatrix: matrix index and row of this lane's address
 #pragma unroll
   for (int s = 0; s < NS - 1; ++s) {
-    issue(t_begin + s, s);
+    issue_next();
     cp_async_commit();
   }
 
+  // compute cursor: tile t, its unit and ring stage
+  int unit = t_begin / p.tiles_per_group, tile_in_unit = t_begin % p.tiles_per_group, st = 0;
   for (int t = t_begin; t < t_end; ++t) {
-    const int st = (t - t_begin) % NS;
-    issue(t + NS - 1, (t + NS - 1 - t_begin) % NS);
+    issue_next();
     cp_async_commit();
     cp_async_wait<NS - 1>();
     __syncwarp();
-    const int unit = t / p.tiles_per_group;
     if (unit != cur_unit) {
       if (cur_unit >= 0) flush(cur_unit);
       start_unit(unit);
@@ -278,6 +286,11 @@ __global__ void __launch_bounds__(MmaLayout<D, NS>::W * 32, 1) attn_mma_kernel(A
       }
     }
     __syncwarp();
+    if (++tile_in_unit == p.tiles_per_group) {
+      tile_in_unit = 0;
+      ++unit;
+    }
+    if (++st == NS) st = 0;
   }
   if (cur_unit >= 0) flush(cur_unit);
   cp_async_wait<0>();
@@ -322,6 +335,7 @@ int attn_mma_warps(const AttnArgs &a) {
 }
 
 cudaError_t launch_attention_mma(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) {
+  if (p.n_head_chunks != 1) return cudaErrorInvalidValue;  // the kernel takes a unit to be a whole group
   if (a.d_qk == 128) return a.paged ? dispatch_mma<128, true>(a, p, st) : dispatch_mma<128, false>(a, p, st);
   return a.paged ? dispatch_mma<64, true>(a, p, st) : dispatch_mma<64, false>(a, p, st);
 }
