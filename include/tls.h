@@ -121,6 +121,23 @@ TLS_API size_t tls_workspace_size(const tls_shape *s);
 TLS_API tls_status tls_build_block_meta(const tls_shape *s, const void *K, const int32_t *seq_lens,
                                 const int32_t *label_idx, void *meta_out, void *slab_out, void *stream);
 
+/* Decode-loop upkeep of the set-up structures: the caller has written the K
+ * rows of tokens [old_lens[b], new_lens[b]) of every sequence b; this rebuilds
+ * the summaries of the blocks those rows fall in (from all their valid rows,
+ * so the result equals tls_build_block_meta at new_lens, bit for bit) and
+ * writes the appended tokens' slab rows (slab_out NULL: summaries only).
+ * gist.science (de) section 2.A "Stufe 1": the per-block max / min summary;
+ * a new decode token only changes the last block's.
+ *   old_lens, new_lens device int32 [B], 0 <= old <= new <= max_ctx
+ *   max_append         host bound on new - old over all b (sizes the launch);
+ *                      a sequence whose range is invalid or longer than
+ *                      max_append is left untouched and sets bit 4 of the
+ *                      device error word (tls_device_error)
+ *   K, label_idx, meta, slab as in tls_build_block_meta. */
+TLS_API tls_status tls_append_tokens(const tls_shape *s, const void *K, const int32_t *old_lens,
+                                     const int32_t *new_lens, int32_t max_append, const int32_t *label_idx,
+                                     void *meta, void *slab, void *stream);
+
 /* Stages 1+2: block bound and top-K_b blocks.
  * gist.science (de) section 2.A "Stufe 1" + "Optimierung", (es) section 2.A.1:
  *   u_{h,j} = sum_i max(q_{h,i} max_{j,i}, q_{h,i} min_{j,i})
@@ -248,8 +265,10 @@ TLS_API tls_status tls_block_score_topk_noalloc(const tls_shape *s, const void *
 /* Device-side failure flags of the current device.  Kernels that wait on
  * other CTAs or on the tensor-core/copy engines bound every wait; when one
  * gives up (which a correct run never sees) the kernel still ends, its outputs
- * are undefined, and it sets a bit in a library-owned device word:
- *   1 = an attention kernel's wait, 2 = a selection cluster's exchange wait.
+ * are undefined, and it sets a bit in a library-owned device word; kernels
+ * that meet an argument only the device can check set a bit there too:
+ *   1 = an attention kernel's wait, 2 = a selection cluster's exchange wait,
+ *   4 = tls_append_tokens got a length range it could not apply.
  * Writes the word to *flags_out (0 = no failure since the last clear) and,
  * when clear != 0, zeroes it.  Reads with a synchronous cudaMemcpy, so call it
  * after the work to check has completed. */

@@ -125,6 +125,15 @@ def test_select_step_checks_before_launch(T):
     assert st == T.TLS_ERR_UNSUPPORTED
 
 
+def test_append_tokens_checks_before_launch(T):
+    s = good_shape(T)
+    assert T._lib.tls_append_tokens(ctypes.byref(s), 256, 256, 256, -1, 256, 256, None, None) == T.TLS_ERR_INVALID_ARG
+    assert "max_append" in T.tls_last_error()
+    assert T._lib.tls_append_tokens(ctypes.byref(s), None, 256, 256, 4, 256, 256, None, None) == T.TLS_ERR_INVALID_ARG
+    assert "K is NULL" in T.tls_last_error()
+    assert T._lib.tls_append_tokens(ctypes.byref(s), None, None, None, 0, None, None, None, None) == T.TLS_OK
+
+
 def test_device_error_checks_its_argument(T):
     assert T._lib.tls_device_error(None, 0) == T.TLS_ERR_INVALID_ARG
     assert "flags_out is NULL" in T.tls_last_error()

@@ -212,6 +212,27 @@ tls_status tls_build_block_meta(const tls_shape *s, const void *K, const int32_t
   return cuda_status(tls::launch_build_slab(a, cs), "build_slab launch");
 }
 
+tls_status tls_append_tokens(const tls_shape *s, const void *K, const int32_t *old_lens, const int32_t *new_lens,
+                             int32_t max_append, const int32_t *label_idx, void *meta, void *slab, void *stream) {
+  tls_status st = check_shape(s);
+  if (st != TLS_OK) return st;
+  if (s->batch == 0 || max_append == 0) return TLS_OK;
+  if (max_append < 0 || max_append > s->max_ctx)
+    return fail(TLS_ERR_INVALID_ARG, "max_append %d outside [0, max_ctx]", max_append);
+  CHECK_PTR(K, 16);
+  CHECK_PTR(old_lens, 4);
+  CHECK_PTR(new_lens, 4);
+  CHECK_PTR(meta, 16);
+  if (slab) {
+    CHECK_PTR(label_idx, 4);
+    CHECK_PTR(slab, 4);
+  }
+  tls::AppendArgs a{{K, nullptr, label_idx, meta, slab, s->batch, s->n_kv_heads, s->d_qk, s->block_size,
+                     n_blocks_max(s), s->max_ctx, s->n_label, s->kv_dtype},
+                    old_lens, new_lens, max_append, tls::device_error_word()};
+  return cuda_status(tls::launch_append_tokens(a, static_cast<cudaStream_t>(stream)), "append_tokens launch");
+}
+
 tls_status tls_block_score_topk(const tls_shape *s, const void *q, const void *meta, const int32_t *seq_lens,
                                 int32_t *block_idx_out, float *block_score_out, void *ws, size_t ws_bytes,
                                 void *stream) {

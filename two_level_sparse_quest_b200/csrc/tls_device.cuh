@@ -265,6 +265,7 @@ __device__ __forceinline__ bool mbarrier_wait_cluster(uint64_t *bar, uint32_t pa
 // gave up; read by tls_device_error).
 constexpr int kErrAttnWait = 1;
 constexpr int kErrSelectWait = 2;
+constexpr int kErrAppendRange = 4;  // an appended range outside [0, max_ctx] or longer than max_append
 
 // ---------------------------------------------------------------- cluster top-k
 //

@@ -62,6 +62,15 @@ struct MetaArgs {
 };
 cudaError_t launch_build_meta(const MetaArgs &a, cudaStream_t st);
 cudaError_t launch_build_slab(const MetaArgs &a, cudaStream_t st);
+// Incremental update after appending tokens [old_lens[b], new_lens[b]) to K:
+// rebuilds the summaries of the blocks those rows fall in and their slab rows.
+struct AppendArgs {
+  MetaArgs m;                 // m.seq_lens unused
+  const int32_t *old_lens, *new_lens;
+  int max_append;
+  int *err;
+};
+cudaError_t launch_append_tokens(const AppendArgs &a, cudaStream_t st);
 
 struct BlockScoreArgs {
   const void *q;

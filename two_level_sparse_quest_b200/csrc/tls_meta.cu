@@ -70,7 +70,84 @@ __global__ void __launch_bounds__(256) build_slab_kernel(MetaArgs a) {
   static_cast<S *>(a.slab)[(static_cast<size_t>(group) * a.max_ctx + t) * a.n_label + c] = v;
 }
 
+// Append update: CTA (j, group) rebuilds the j-th block touched by the rows
+// [old, new) of the group's sequence from the block's valid rows (max / min
+// over the stored values: exact, so the result equals a rebuild at the new
+// length) and writes the slab rows of the appended tokens in that block.
+template <typename E>
+__global__ void __launch_bounds__(128) append_tokens_kernel(AppendArgs a) {
+  grid_dependency_wait();
+  using S = typename E::storage;
+  constexpr int EPC = E::kEPC;
+  const MetaArgs &m = a.m;
+  const int group = blockIdx.y;
+  const int b = group / m.n_kv_heads;
+  const int old_len = a.old_lens[b], new_len = a.new_lens[b];
+  if (old_len < 0 || new_len < old_len || new_len > m.max_ctx || new_len - old_len > a.max_append) {
+    if (blockIdx.x == 0 && threadIdx.x == 0 && a.err) atomicOr(a.err, kErrAppendRange);
+    return;
+  }
+  if (new_len == old_len) return;
+  const int bs = m.block_size;
+  const int blk = old_len / bs + static_cast<int>(blockIdx.x);
+  const int t0 = blk * bs;
+  if (t0 >= new_len) return;
+  const int t1 = min(t0 + bs, new_len);
+  const S *K = static_cast<const S *>(m.K) + static_cast<size_t>(group) * m.max_ctx * m.d;
+  // block summary: one thread per 16-byte chunk of the channels
+  const int chunks = m.d / EPC;
+  S *mo = static_cast<S *>(m.meta) + ((static_cast<size_t>(group) * m.n_blocks_max + blk) * 2) * m.d;
+  for (int c = threadIdx.x; c < chunks; c += blockDim.x) {
+    float hi[EPC], lo[EPC];
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) {
+      hi[e] = -INFINITY;
+      lo[e] = INFINITY;
+    }
+    for (int t = t0; t < t1; ++t) {
+      uint4 v = ld_stream16(K + static_cast<size_t>(t) * m.d + c * EPC);
+      float f[EPC];
+      chunk_to_f32<E>(v, f);
+#pragma unroll
+      for (int e = 0; e < EPC; ++e) {
+        hi[e] = fmaxf(hi[e], f[e]);
+        lo[e] = fminf(lo[e], f[e]);
+      }
+    }
+    S ho[EPC], lw[EPC];
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) {
+      if constexpr (sizeof(S) == 2) {
+        ho[e] = static_cast<S>(__float_as_uint(hi[e]) >> 16);  // exact: the value came from a bf16
+        lw[e] = static_cast<S>(__float_as_uint(lo[e]) >> 16);
+      } else {
+        ho[e] = hi[e];
+        lw[e] = lo[e];
+      }
+    }
+    *reinterpret_cast<uint4 *>(mo + c * EPC) = *reinterpret_cast<const uint4 *>(ho);
+    *reinterpret_cast<uint4 *>(mo + m.d + c * EPC) = *reinterpret_cast<const uint4 *>(lw);
+  }
+  // label slab rows of the appended tokens in this block
+  if (m.slab) {
+    const int s0 = max(t0, old_len);
+    S *slab = static_cast<S *>(m.slab) + static_cast<size_t>(group) * m.max_ctx * m.n_label;
+    for (int i = threadIdx.x; i < (t1 - s0) * m.n_label; i += blockDim.x) {
+      const int t = s0 + i / m.n_label, c = i % m.n_label;
+      const int ch = m.label_idx[c];
+      slab[static_cast<size_t>(t) * m.n_label + c] = (ch >= 0 && ch < m.d) ? K[static_cast<size_t>(t) * m.d + ch] : S(0);
+    }
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_append_tokens(const AppendArgs &a, cudaStream_t st) {
+  const int nblk = (a.max_append + a.m.block_size - 1) / a.m.block_size + 1;  // blocks one range can touch
+  dim3 grid(static_cast<unsigned>(nblk), a.m.batch * a.m.n_kv_heads);
+  if (a.m.dtype == 1) return launch_pdl(append_tokens_kernel<BF16>, grid, dim3(128), 0, st, a);
+  return launch_pdl(append_tokens_kernel<F32>, grid, dim3(128), 0, st, a);
+}
 
 cudaError_t launch_build_meta(const MetaArgs &a, cudaStream_t st) {
   const int epc = a.dtype == 1 ? BF16::kEPC : F32::kEPC;

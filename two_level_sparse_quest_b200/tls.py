@@ -30,7 +30,8 @@ STATUS_NAMES = {0: "TLS_OK", 1: "TLS_ERR_INVALID_ARG", 2: "TLS_ERR_UNSUPPORTED",
 
 EXPORTED = ("tls_version", "tls_last_error", "tls_workspace_size", "tls_build_block_meta", "tls_block_score_topk",
             "tls_token_score_topk", "tls_sparse_attn_decode", "tls_sparse_attn_decode_paged", "tls_offload_reset",
-            "tls_prefetch_diff", "tls_wait_event", "tls_block_score_topk_noalloc", "tls_device_error", "tls_select_step")
+            "tls_prefetch_diff", "tls_wait_event", "tls_block_score_topk_noalloc", "tls_device_error", "tls_select_step",
+            "tls_append_tokens")
 
 
 class TlsShape(ctypes.Structure):
@@ -67,6 +68,7 @@ _sigs = {
     "tls_block_score_topk_noalloc": ([_S, _P, _P, _P, _P, _P], ctypes.c_int),
     "tls_device_error": ([ctypes.POINTER(_i32), _i32], ctypes.c_int),
     "tls_select_step": ([_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
+    "tls_append_tokens": ([_S, _P, _P, _P, _i32, _P, _P, _P, _P], ctypes.c_int),
 }
 for _name, (_args, _ret) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -144,6 +146,12 @@ def tls_workspace_size(shape: TlsShape) -> int:
 def tls_build_block_meta(shape, K, seq_lens, label_idx, meta_out, slab_out=None, stream=None):
     _check(_lib.tls_build_block_meta(ctypes.byref(shape), _ptr(K), _ptr(seq_lens), _ptr(label_idx), _ptr(meta_out),
                                      _ptr(slab_out), _stream(stream)), "tls_build_block_meta")
+
+
+def tls_append_tokens(shape, K, old_lens, new_lens, max_append, label_idx, meta_out, slab_out=None, stream=None):
+    _check(_lib.tls_append_tokens(ctypes.byref(shape), _ptr(K), _ptr(old_lens), _ptr(new_lens), int(max_append),
+                                  _ptr(label_idx), _ptr(meta_out), _ptr(slab_out), _stream(stream)),
+           "tls_append_tokens")
 
 
 def tls_block_score_topk(shape, q, meta, seq_lens, block_idx_out, block_score_out=None, ws=None, stream=None):
