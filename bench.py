@@ -474,6 +474,53 @@ def offload_arm(args):
     }
 
 
+# ----------------------------------------------------------------------------- dense context
+def dense_arm(args):
+    """Full-attention decode of the same workload on the same GPU, for context:
+    the attention kernels with every token of every sequence selected (K_t = n),
+    so each step streams the whole K/V cache once.  Reports its time per step
+    next to the sparse step's (measured the same way)."""
+    import numpy as np
+    import torch
+
+    from two_level_sparse_quest_b200 import build as tls_build
+
+    tls_build.build()
+    from two_level_sparse_quest_b200 import tls as T
+    from two_level_sparse_quest_b200 import workloads as W
+
+    dev = torch.device("cuda", 0)
+    w = W.WORKLOADS[args.workload]
+    inp = W.make_decode_inputs(w)
+
+    def up(a):
+        return torch.from_numpy(np.ascontiguousarray(a.view(np.int16) if a.dtype == np.uint16 else a)).to(dev)
+
+    q, K = up(inp.q), up(inp.K)
+    V = up(inp.V) if inp.V is not None else None
+    G = w.batch * w.n_kv_heads
+    dense = T.shape_from_workload(w, k_t=w.ctx)
+    all_tok = torch.arange(w.ctx, dtype=torch.int32, device=dev).repeat(G, 1).contiguous()
+    ws = torch.zeros(T.tls_workspace_size(dense), dtype=torch.uint8, device=dev)
+    out = torch.empty((w.batch, w.n_q_heads, w.d_v), dtype=torch.float32, device=dev)
+    lse = torch.empty((w.batch, w.n_q_heads), dtype=torch.float32, device=dev)
+    steps = max(3, min(args.steps, 50))
+    for _ in range(3):
+        T.tls_sparse_attn_decode(dense, q, K, V, all_tok, out, lse, ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        T.tls_sparse_attn_decode(dense, q, K, V, all_tok, out, lse, ws)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / steps
+    kv_bytes = G * w.ctx * (w.d_qk + (0 if w.v_is_k_prefix else w.d_v)) * w.elem_bytes
+    return {"metric": "dense decode attention (all tokens) per step, same kernels", "workload": args.workload,
+            "dense_us_per_step": ms * 1e3, "dense_kv_bytes": kv_bytes, "dense_gbs": kv_bytes / (ms * 1e-3) / 1e9,
+            "steps": steps, "input": "the whole cache is larger than L2, so no rotation is needed"}
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def oracle_sample(args, budget_s: float):
     """The fp64 oracle (single thread) on a bounded sample of the workload: the
@@ -536,6 +583,8 @@ def main():
     ap.add_argument("--workload", default="gqa96k_b8_bf16")
     ap.add_argument("--impl", default="tls", choices=["tls", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dense", action="store_true",
+                    help="time full-attention decode (all tokens selected) of the workload, for context")
     ap.add_argument("--offload", action="store_true",
                     help="time the offload engine on the streaming workload instead (one JSON line of its own)")
     ap.add_argument("--layers", type=int, default=N_LAYERS_DEFAULT,
@@ -547,6 +596,11 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.dense:
+        if rank == 0:
+            print(json.dumps(dense_arm(args)), flush=True)
+        return
 
     if args.offload:
         if rank == 0:
