@@ -104,3 +104,26 @@ def test_full_size_parity(name):
     # spec: index sets bit-exact except counted boundary swaps
     assert res["block_swaps"] <= max(1, res["groups"] // 8)
     assert res["token_swaps"] <= max(1, res["groups"] // 8)
+
+
+@pytest.mark.parametrize("impl", ["cuda_core", "tensor_core"])
+def test_alternative_attention_kernels_parity(impl):
+    """The attention kernels that TLS_ATTN_IMPL selects instead of the default
+    (read once per process, so each runs in a child process): the CUDA-core
+    kernel for GQA bf16 and latent shapes, the tcgen05 kernel for GQA bf16."""
+    import os
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cases = ["gqa_bf16_small", "gqa_bf16_g8", "mla_small"] if impl == "cuda_core" else ["gqa_bf16_small", "gqa_bf16_g8"]
+    code = (
+        "import sys; sys.path.insert(0, %r)\n"
+        "from tests import test_gpu_parity as t, _parity as P\n"
+        "for n in %r:\n"
+        "    w, sl = t.SMALL[n]\n"
+        "    P.full_stage_parity(w, seq_lens=sl, name=n + ':' + %r)\n"
+        "print('ok')\n" % (root, cases, impl))
+    env = dict(os.environ, TLS_ATTN_IMPL=impl)
+    r = subprocess.run([sys.executable, "-c", code], env=env, cwd=root, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout[-2000:] + r.stderr[-4000:]

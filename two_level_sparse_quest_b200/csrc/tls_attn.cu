@@ -415,10 +415,11 @@ cudaError_t dispatch_gqa(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) 
 }  // namespace
 
 // Kernel choice.  bf16 GQA shapes run the warp-MMA kernel (tls_attn_mma.cu)
-// by default; TLS_ATTN_IMPL=cuda_core selects this file's CUDA-core kernel and
-// TLS_ATTN_IMPL=tensor_core the tcgen05 kernel (bf16, d = 128) instead.  The
-// variable is read once per process.  Other shapes (fp32, latent attention)
-// always run the CUDA-core kernel.
+// and latent shapes with 16, 32 or 64 heads the warp-MMA latent kernel
+// (tls_attn_mla.cu) by default; TLS_ATTN_IMPL=cuda_core selects this file's
+// CUDA-core kernel for both, TLS_ATTN_IMPL=tensor_core the tcgen05 kernel
+// (bf16 GQA, d = 128).  The variable is read once per process.  fp32 shapes
+// and other latent head counts always run the CUDA-core kernel.
 enum ImplChoice { kImplDefault = 0, kImplCudaCore = 1, kImplTcgen05 = 2 };
 static int impl_choice() {
   static int choice = -1;
@@ -436,6 +437,28 @@ bool attn_plan(const AttnArgs &a, AttnPlan *p) {
   if (choice == kImplTcgen05 && attn_tc_supported(a)) {
     p->impl = 1;
     return attn_tc_plan(a, p);
+  }
+  if (choice == kImplDefault && attn_mla_supported(a)) {
+    // latent attention on the tensor cores: a unit is a whole group (all G
+    // heads), a piece is one CTA's contiguous range of 16-token tiles
+    const int G = a.n_q_heads / a.n_kv_heads;
+    p->impl = 3;
+    p->warps_per_cta = 8;
+    p->tokens_per_tile = 16;
+    p->head_chunk = G;
+    p->n_head_chunks = 1;
+    const long long units = static_cast<long long>(a.batch) * a.n_kv_heads;
+    p->tiles_per_group = (a.k_t + 15) / 16;
+    const long long total = units * p->tiles_per_group;
+    if (total <= 0 || total > (1LL << 30)) return false;
+    p->total_tiles = static_cast<int>(total);
+    const int sms = a.num_sms > 0 ? a.num_sms : 148;
+    const long long g0 = std::min<long long>(sms, total);
+    p->tiles_per_warp = static_cast<int>((total + g0 - 1) / g0);
+    p->grid = static_cast<int>((total + p->tiles_per_warp - 1) / p->tiles_per_warp);
+    p->max_pieces = (p->tiles_per_group + p->tiles_per_warp - 1) / p->tiles_per_warp + 1;
+    p->part_floats = static_cast<size_t>(units) * p->max_pieces * G * (2 + a.d_v);
+    return true;
   }
   const bool mma = choice == kImplDefault && attn_mma_supported(a);
   p->impl = mma ? 2 : 0;
@@ -464,6 +487,7 @@ bool attn_plan(const AttnArgs &a, AttnPlan *p) {
 static cudaError_t launch_split(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) {
   if (p.impl == 1) return launch_attention_tc(a, p, st);
   if (p.impl == 2) return launch_attention_mma(a, p, st);
+  if (p.impl == 3) return launch_attention_mla(a, p, st);
   if (a.v_is_k_prefix) return run_attention<BF16, 576, 512, 4, true, false, kStages>(a, p, st);
   if (a.dtype == 1) {
     if (a.d_qk == 128) return a.paged ? dispatch_gqa<BF16, 128, true>(a, p, st) : dispatch_gqa<BF16, 128, false>(a, p, st);
@@ -474,7 +498,17 @@ static cudaError_t launch_split(const AttnArgs &a, const AttnPlan &p, cudaStream
 }
 
 cudaError_t launch_attention_merge(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) {
-  if (a.v_is_k_prefix) return run_merge<512, 4>(a, p, st);
+  if (a.v_is_k_prefix) {
+    if (p.impl == 3) {
+      switch (p.head_chunk) {
+        case 16: return run_merge<512, 16>(a, p, st);
+        case 32: return run_merge<512, 32>(a, p, st);
+        case 64: return run_merge<512, 64>(a, p, st);
+      }
+      return cudaErrorInvalidValue;
+    }
+    return run_merge<512, 4>(a, p, st);
+  }
   const int dv = a.d_v;
   switch (p.head_chunk) {
     case 1: return dv == 128 ? run_merge<128, 1>(a, p, st) : run_merge<64, 1>(a, p, st);

@@ -119,7 +119,8 @@ struct AttnArgs {
 // Partial-result layout chosen for a shape on a device; shared by the
 // workspace query and the launch so both agree.
 struct AttnPlan {
-  int impl;  // 0: CUDA-core kernel, 1: tcgen05 kernel (tiles_per_warp counts tiles per CTA), 2: warp-MMA kernel
+  int impl;  // 0: CUDA-core kernel, 1: tcgen05 kernel, 2: warp-MMA GQA kernel, 3: warp-MMA latent kernel
+             // (for 1 and 3 tiles_per_warp counts tiles per CTA)
   int warps_per_cta, tokens_per_tile, head_chunk, n_head_chunks;
   int tiles_per_group, total_tiles, grid, tiles_per_warp, max_pieces;
   size_t part_floats;  // floats of workspace for partials
@@ -127,6 +128,8 @@ struct AttnPlan {
 bool attn_plan(const AttnArgs &a, AttnPlan *p);
 cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &p, cudaStream_t st);
 // tensor-core (tcgen05) attention for GQA bf16 d = 128
+bool attn_mla_supported(const AttnArgs &a);
+cudaError_t launch_attention_mla(const AttnArgs &a, const AttnPlan &p, cudaStream_t st);
 bool attn_mma_supported(const AttnArgs &a);
 int attn_mma_warps(const AttnArgs &a);
 cudaError_t launch_attention_mma(const AttnArgs &a, const AttnPlan &p, cudaStream_t st);
