@@ -82,6 +82,8 @@ typedef struct tls_shape {
   int32_t kv_dtype;      /* tls_dtype of q, K, V, meta, slab and cache                   */
   int32_t out_dtype;     /* tls_dtype of the attention output                            */
   float softmax_scale;   /* tau; <= 0 selects 1/sqrt(d_qk)                               */
+  int32_t block_agg;     /* block score over the group's heads: 0 = sum of the heads'
+                          * bounds (the method), 1 = their maximum (a variant; GQA only)  */
 } tls_shape;
 
 /* Supported shapes (others return TLS_ERR_UNSUPPORTED):

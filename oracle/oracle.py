@@ -27,7 +27,7 @@ _lib = None
 class OraShape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "batch", "n_q_heads", "n_kv_heads", "d_qk", "d_v", "v_is_k_prefix",
-        "block_size", "n_label", "k_b", "k_t", "max_ctx", "dtype")] + [("softmax_scale", ctypes.c_double)]
+        "block_size", "n_label", "k_b", "k_t", "max_ctx", "dtype", "block_agg")] + [("softmax_scale", ctypes.c_double)]
 
 
 def build(force: bool = False) -> str:
@@ -73,6 +73,7 @@ def shape_of(w, k_b: Optional[int] = None, k_t: Optional[int] = None, softmax_sc
     s.k_b = w.k_b if k_b is None else k_b
     s.k_t = w.k_t if k_t is None else k_t
     s.max_ctx, s.dtype = w.ctx, w.dtype
+    s.block_agg = int(getattr(w, "block_agg", 0))
     s.softmax_scale = (1.0 / math.sqrt(w.d_qk)) if softmax_scale is None else softmax_scale
     return s
 

@@ -34,6 +34,7 @@
 typedef struct {
   int batch, n_q_heads, n_kv_heads, d_qk, d_v, v_is_k_prefix;
   int block_size, n_label, k_b, k_t, max_ctx, dtype; /* dtype 0: fp32, 1: bf16 bits */
+  int block_agg;                                      /* 0: sum of the heads' bounds, 1: their max */
   double softmax_scale;
 } ora_shape;
 
@@ -86,7 +87,9 @@ void ora_build_meta(const ora_shape *s, const void *K, const int32_t *seq_lens, 
  * key k inside the box [min_j, max_j] is
  *     u_{h,j} = sum_i max(q_{h,i} * max_{j,i}, q_{h,i} * min_{j,i}).
  * The heads sharing one KV head (GQA) or one latent (MLA) share one selection;
- * their bounds are added:  score_j = sum_{h in group} u_{h,j}.
+ * their bounds are added:  score_j = sum_{h in group} u_{h,j}  (block_agg 0),
+ * or, as the variant, the largest one is taken: score_j = max_h u_{h,j}
+ * (block_agg 1).
  * score: [B][H_kv][N_b_max]; blocks at or beyond ceil(seq_len / bs) get -inf. */
 void ora_block_scores(const ora_shape *s, const void *q, const double *meta, const int32_t *seq_lens,
                       double *score) {
@@ -99,7 +102,7 @@ void ora_block_scores(const ora_shape *s, const void *q, const double *meta, con
         if (j >= nb) { *out = -INFINITY; continue; }
         const double *mx = meta + ((((size_t)b * s->n_kv_heads + g) * nbm + j) * 2) * d;
         const double *mn = mx + d;
-        double total = 0.0;
+        double total = s->block_agg ? -INFINITY : 0.0;
         for (int hh = 0; hh < G; ++hh) {
           const int h = g * G + hh;
           double u = 0.0;
@@ -108,7 +111,8 @@ void ora_block_scores(const ora_shape *s, const void *q, const double *meta, con
             double a = qi * mx[i], c = qi * mn[i];
             u += (a > c) ? a : c;
           }
-          total += u;
+          if (s->block_agg) total = (u > total) ? u : total;
+          else total += u;
         }
         *out = total;
       }

@@ -116,6 +116,15 @@ def test_pointer_checks(T):
     assert st == T.TLS_ERR_WORKSPACE
 
 
+def test_block_aggregation_field_is_checked(T):
+    s = good_shape(T)
+    s.block_agg = 2
+    assert call_block(T, s) == T.TLS_ERR_INVALID_ARG and "block_agg" in T.tls_last_error()
+    mla = good_shape(T, v_is_k_prefix=True, n_q_heads=64, n_kv_heads=1, d_qk=576, d_v=512, n_label=32)
+    mla.block_agg = 1
+    assert call_block(T, mla) == T.TLS_ERR_UNSUPPORTED
+
+
 def test_select_step_checks_before_launch(T):
     s = good_shape(T)
     st = T._lib.tls_select_step(ctypes.byref(s), 256, 256, None, 256, 256, 256, 256, None, None, None)

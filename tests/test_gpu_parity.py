@@ -95,6 +95,37 @@ def test_tie_heavy_selection_parity(name):
     P().full_stage_parity(w, name=name, inp=inp)
 
 
+AGG_MAX = {
+    # the max-over-heads block aggregation variant, through the separate stages
+    "agg_max_bf16_g4": (W.WORKLOADS["gqa48k_bf16"].with_(batch=2, ctx=4096, k_b=24, k_t=300, block_agg=1),
+                        [4096, 3001]),
+    "agg_max_f32_ragged": (W.WORKLOADS["tiny_gqa4k_f32"].with_(batch=3, ctx=1000, k_b=8, k_t=100, n_q_heads=8,
+                                                                block_agg=1), [1000, 777, 33]),
+    "agg_max_full_gqa96k_b8": (W.WORKLOADS["gqa96k_b8_bf16"].with_(block_agg=1), None),
+}
+
+
+@pytest.mark.parametrize("name", sorted(AGG_MAX))
+def test_max_aggregation_variant_parity(name):
+    w, sl = AGG_MAX[name]
+    res = P().full_stage_parity(w, seq_lens=sl, name=name)
+    assert res["block_swaps"] <= max(1, res["groups"] // 8)
+
+
+def test_max_aggregation_select_step_equals_separate_calls():
+    from tests import _parity as PP
+    from two_level_sparse_quest_b200 import tls as T
+
+    w = W.WORKLOADS["gqa48k_bf16"].with_(batch=2, ctx=4096, k_b=24, k_t=300, block_agg=1)
+    g = PP.GpuInputs(w, W.make_decode_inputs(w))
+    bidx, _ = g.block_stage()
+    tidx, _ = g.token_stage(bidx)
+    fb, ft = torch.full_like(bidx, -7), torch.full_like(tidx, -7)
+    T.tls_select_step(g.shape, g.q, g.meta, g.slab, g.label, g.seq_lens, fb, ft)
+    torch.cuda.synchronize()
+    assert torch.equal(fb, bidx) and torch.equal(ft, tidx)
+
+
 FULL = ["tiny_gqa4k_f32", "gqa48k_bf16", "gqa96k_b8_bf16", "mla64k_b4_bf16"]
 
 

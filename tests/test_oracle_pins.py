@@ -111,6 +111,29 @@ def test_block_bound_dominates_every_key(seed):
                 assert score[b, g, j] >= dots.sum(axis=0).max() - 1e-12
 
 
+@pytest.mark.parametrize("seed", [0, 1])
+def test_max_over_heads_aggregation_is_the_largest_single_head_bound(seed):
+    """The aggregation variant: a group's block score is the largest of its
+    heads' bounds, each obtained by running the oracle on that head alone; with
+    one head per group both aggregations coincide."""
+    sh = Sh(batch=2, n_q_heads=8, n_kv_heads=2, ctx=48, block_size=8, d_qk=6)
+    q, K, V, sl = rand_inputs(sh, seed, seq_lens=[48, 21])
+    meta = O.build_meta(O.shape_of(sh), K, sl)
+    shm = Sh(**{**sh.__dict__, "block_agg": 1})
+    smax = O.block_scores(O.shape_of(shm), q, meta, sl)
+    ssum = O.block_scores(O.shape_of(sh), q, meta, sl)
+    u = per_head_bounds(sh, q, meta, sl)  # [B][H_q][N_b]
+    G = sh.n_q_heads // sh.n_kv_heads
+    want = u.reshape(sh.batch, sh.n_kv_heads, G, -1).max(axis=2)
+    np.testing.assert_array_equal(smax, want)
+    assert not np.array_equal(np.nan_to_num(smax, neginf=0), np.nan_to_num(ssum, neginf=0))
+    one = Sh(**{**sh.__dict__, "n_q_heads": 2, "n_kv_heads": 2})
+    one_max = Sh(**{**one.__dict__, "block_agg": 1})
+    q1 = np.ascontiguousarray(q[:, :2])
+    np.testing.assert_array_equal(O.block_scores(O.shape_of(one), q1, meta, sl),
+                                  O.block_scores(O.shape_of(one_max), q1, meta, sl))
+
+
 def test_block_bound_is_attained_at_box_corner():
     # max of a linear function over a box is attained at the corner that follows sign(q)
     sh = Sh(n_q_heads=1, n_kv_heads=1, ctx=64, block_size=16, d_qk=9)

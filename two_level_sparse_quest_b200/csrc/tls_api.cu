@@ -67,6 +67,9 @@ tls_status check_shape(const tls_shape *s) {
   if (s->k_b < 1 || s->k_t < 1) return fail(TLS_ERR_INVALID_ARG, "k_b and k_t must be >= 1");
   if (s->d_qk < 1 || s->d_v < 1) return fail(TLS_ERR_INVALID_ARG, "d_qk and d_v must be >= 1");
   if (s->v_is_k_prefix && s->d_v > s->d_qk) return fail(TLS_ERR_INVALID_ARG, "v_is_k_prefix needs d_v <= d_qk");
+  if (s->block_agg != 0 && s->block_agg != 1) return fail(TLS_ERR_INVALID_ARG, "block_agg %d", s->block_agg);
+  if (s->block_agg == 1 && s->v_is_k_prefix)
+    return fail(TLS_ERR_UNSUPPORTED, "max-over-heads block aggregation supports GQA shapes only");
   if (static_cast<long long>(s->batch) * s->n_kv_heads > 65535)
     return fail(TLS_ERR_UNSUPPORTED, "batch * n_kv_heads > 65535");
   const int G = s->n_q_heads / s->n_kv_heads;
@@ -248,7 +251,7 @@ tls_status tls_block_score_topk(const tls_shape *s, const void *q, const void *m
   (void)ws_bytes;
   tls::BlockScoreArgs a{q, meta, seq_lens, block_score_out, block_idx_out, s->batch, s->n_q_heads, s->n_kv_heads,
                         s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->k_b, s->kv_dtype,
-                        tls::device_error_word()};
+                        tls::device_error_word(), s->block_agg};
   return cuda_status(tls::launch_block_select(a, static_cast<cudaStream_t>(stream)), "block_select launch");
 }
 
@@ -290,11 +293,17 @@ tls_status tls_select_step(const tls_shape *s, const void *q, const void *meta, 
   if (token_score_out && !aligned(token_score_out, 4)) return fail(TLS_ERR_INVALID_ARG, "token_score_out misaligned");
   int *err = tls::device_error_word();
   tls::BlockScoreArgs a{q, meta, seq_lens, block_score_out, block_idx_out, s->batch, s->n_q_heads, s->n_kv_heads,
-                        s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->k_b, s->kv_dtype, err};
+                        s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->k_b, s->kv_dtype, err, s->block_agg};
   tls::TokenArgs t{q, slab, label_idx, block_idx_out, seq_lens, token_idx_out, token_score_out, s->batch, s->n_q_heads,
                    s->n_kv_heads, s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->n_label, s->k_b, s->k_t,
                    s->kv_dtype, err};
-  return cuda_status(tls::launch_select_step(a, t, static_cast<cudaStream_t>(stream)), "select_step launch");
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (s->block_agg == 1) {  // the max-over-heads variant runs as the two separate launches
+    st = cuda_status(tls::launch_block_select(a, cs), "block_select launch");
+    if (st != TLS_OK) return st;
+    return cuda_status(tls::launch_token_select(t, cs), "token_select launch");
+  }
+  return cuda_status(tls::launch_select_step(a, t, cs), "select_step launch");
 }
 
 static tls_status attn_common(const tls_shape *s, const void *q, const void *K, const void *V,

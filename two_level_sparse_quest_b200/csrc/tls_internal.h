@@ -80,6 +80,7 @@ struct BlockScoreArgs {
   int32_t *block_idx; // [B*H_kv][k_b]
   int batch, n_q_heads, n_kv_heads, d, block_size, n_blocks_max, max_ctx, k_b, dtype;
   int *err;           // the library's device error word
+  int agg;            // 0: sum of the heads' bounds, 1: their max
 };
 // Block score and top-K_b in one launch (one thread-block cluster per group).
 cudaError_t launch_block_select(const BlockScoreArgs &a, cudaStream_t st);

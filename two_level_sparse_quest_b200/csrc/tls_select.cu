@@ -130,6 +130,73 @@ __device__ __forceinline__ void score_blocks(const BlockScoreArgs &a, int group,
   }
 }
 
+// The max-over-heads variant of the stage-1 body: qh = [q_h^+; q_h^-] per head
+// (G x 2d floats), every head's bound per row, the largest one is the score.
+// GQA shapes only (G <= 8).
+template <typename E, int NCH>
+__device__ __forceinline__ void score_blocks_max(const BlockScoreArgs &a, int group, int nb, int r0, int r1,
+                                                 float *qh, uint32_t *keys, int *hist) {
+  constexpr int EPC = E::kEPC;
+  constexpr int LPR = NCH < 32 ? NCH : 32;
+  constexpr int RPW = 32 / LPR;
+  constexpr int CPL = (NCH + 31) / 32;
+  constexpr int NWARP = kThreads / 32;
+  constexpr int STEP = NWARP * RPW;
+  constexpr int MAXG = 8;
+  const int b = group / a.n_kv_heads, g = group % a.n_kv_heads;
+  const int G = a.n_q_heads / a.n_kv_heads;
+  const int d = a.d;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int sub = lane / LPR, cl = lane % LPR;
+  const char *meta = static_cast<const char *>(a.meta) + static_cast<size_t>(group) * a.n_blocks_max * (NCH * 16);
+  float *out = a.scores ? a.scores + static_cast<size_t>(group) * a.n_blocks_max : nullptr;
+  for (int i = threadIdx.x; i < G * d; i += kThreads) {
+    const int hh = i / d, c = i % d;
+    const float x = load_elem<E>(a.q, (static_cast<size_t>(b) * a.n_q_heads + g * G + hh) * d + c);
+    qh[hh * 2 * d + c] = fmaxf(x, 0.f);
+    qh[hh * 2 * d + d + c] = fminf(x, 0.f);
+  }
+  __syncthreads();
+  for (int rb = r0 + warp * RPW; rb < r1; rb += STEP) {
+    const int row = rb + sub;
+    const bool ok = row < r1 && row < nb;
+    float acc[MAXG];
+#pragma unroll
+    for (int h = 0; h < MAXG; ++h) acc[h] = 0.f;
+#pragma unroll
+    for (int j = 0; j < CPL; ++j) {
+      const int c = cl + j * 32;
+      if (c < NCH) {
+        const uint4 v = ok ? ld_stream16(meta + static_cast<size_t>(row) * (NCH * 16) + c * 16) : make_uint4(0, 0, 0, 0);
+        float f[EPC];
+        chunk_to_f32<E>(v, f);
+#pragma unroll
+        for (int h = 0; h < MAXG; ++h)
+          if (h < G) {
+            const float *qp = qh + h * 2 * d + c * EPC;
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) acc[h] = fmaf(qp[e], f[e], acc[h]);
+          }
+      }
+    }
+    float best = -INFINITY;
+#pragma unroll
+    for (int h = 0; h < MAXG; ++h) {
+      float x = acc[h];
+#pragma unroll
+      for (int o = LPR / 2; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+      if (h < G) best = fmaxf(best, x);
+    }
+    if (cl == 0 && row < r1) {
+      const bool valid = row < nb;
+      const uint32_t key = valid ? max(score_key(best), 1u) : 0u;
+      keys[row - r0] = key;
+      hist_add(hist, key, valid);
+      if (out) out[row] = valid ? best : -INFINITY;
+    }
+  }
+}
+
 // Qbar_L[c] = sum_h q_h[L[c]] (fp32, heads in order) into qbar[0..r).
 template <typename E>
 __device__ __forceinline__ void fold_label_query(const TokenArgs &a, int group, float *qbar) {
@@ -222,14 +289,15 @@ __device__ __forceinline__ TokenSlice token_slice(const TokenArgs &a, int rank, 
 
 // ---------------------------------------------------------------- kernels
 // grid = (CS, groups), cluster = (CS, 1, 1) for all three.
-template <typename E, int NCH, int CS>
+template <typename E, int NCH, int CS, bool AGG_MAX>
 __global__ void __launch_bounds__(kThreads, NCH > 32 ? 2 : 4) block_select_kernel(BlockScoreArgs a, int rows_per_cta) {
-  extern __shared__ float qpm[];  // [2d]: Q^+ then Q^-, then the slice's keys
+  extern __shared__ float qpm[];  // [2d] Q^+, Q^- (max variant: [G][2d] per head), then the slice's keys
   __shared__ ClusterSelectSmem<CS> S;
   cluster_topk_begin(S);
   const int group = blockIdx.y;
   const int rank = static_cast<int>(cluster_ctarank());
-  uint32_t *keys = reinterpret_cast<uint32_t *>(qpm + 2 * a.d);
+  const int G = a.n_q_heads / a.n_kv_heads;
+  uint32_t *keys = reinterpret_cast<uint32_t *>(qpm + (AGG_MAX ? G : 1) * 2 * a.d);
   if (threadIdx.x < kCBins) S.hist[threadIdx.x] = 0;
   grid_dependency_wait();
   const int b = group / a.n_kv_heads;
@@ -237,7 +305,8 @@ __global__ void __launch_bounds__(kThreads, NCH > 32 ? 2 : 4) block_select_kerne
   const int nb = (sq + a.block_size - 1) / a.block_size;
   const int r0 = rank * rows_per_cta;
   const int r1 = min(r0 + rows_per_cta, a.n_blocks_max);
-  score_blocks<E, NCH>(a, group, nb, r0, r1, qpm, keys, S.hist);
+  if constexpr (AGG_MAX) score_blocks_max<E, NCH>(a, group, nb, r0, r1, qpm, keys, S.hist);
+  else score_blocks<E, NCH>(a, group, nb, r0, r1, qpm, keys, S.hist);
   cluster_topk<kThreads, CS, kSliceCap>(
       keys, max(r1 - r0, 0), a.k_b, a.block_idx + static_cast<size_t>(group) * a.k_b, a.k_b,
       [r0](int i) { return r0 + i; }, S, a.err);
@@ -348,16 +417,26 @@ cudaError_t allow_smem(K kern, size_t bytes, int (&allowed)[64]) {
   return e;
 }
 
-template <typename E, int NCH>
-cudaError_t run_block_select(const BlockScoreArgs &a, cudaStream_t st) {
+template <typename E, int NCH, bool AGG_MAX>
+cudaError_t run_block_select_agg(const BlockScoreArgs &a, cudaStream_t st) {
   constexpr int CS = kClusterSize;
   const int rows = (a.n_blocks_max + CS - 1) / CS;  // <= kSliceCap
-  const size_t smem = 2 * static_cast<size_t>(a.d) * sizeof(float) + static_cast<size_t>(rows) * sizeof(uint32_t);
+  const int qrows = AGG_MAX ? a.n_q_heads / a.n_kv_heads : 1;
+  const size_t smem =
+      static_cast<size_t>(qrows) * 2 * a.d * sizeof(float) + static_cast<size_t>(rows) * sizeof(uint32_t);
   static int allowed[64] = {};
-  cudaError_t e = allow_smem(block_select_kernel<E, NCH, CS>, smem, allowed);
+  cudaError_t e = allow_smem(block_select_kernel<E, NCH, CS, AGG_MAX>, smem, allowed);
   if (e != cudaSuccess) return e;
-  return launch_pdl_cluster(block_select_kernel<E, NCH, CS>, dim3(CS, a.batch * a.n_kv_heads), dim3(kThreads), smem,
-                            st, CS, a, rows);
+  return launch_pdl_cluster(block_select_kernel<E, NCH, CS, AGG_MAX>, dim3(CS, a.batch * a.n_kv_heads),
+                            dim3(kThreads), smem, st, CS, a, rows);
+}
+template <typename E, int NCH>
+cudaError_t run_block_select(const BlockScoreArgs &a, cudaStream_t st) {
+  if (a.agg == 1) {
+    if constexpr (NCH <= 64) return run_block_select_agg<E, NCH, true>(a, st);
+    return cudaErrorInvalidValue;  // latent shapes: max aggregation not offered
+  }
+  return run_block_select_agg<E, NCH, false>(a, st);
 }
 
 template <typename E, int RCH>

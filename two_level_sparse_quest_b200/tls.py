@@ -37,7 +37,8 @@ EXPORTED = ("tls_version", "tls_last_error", "tls_workspace_size", "tls_build_bl
 class TlsShape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "batch", "n_q_heads", "n_kv_heads", "d_qk", "d_v", "v_is_k_prefix", "block_size", "n_label",
-        "k_b", "k_t", "max_ctx", "kv_dtype", "out_dtype")] + [("softmax_scale", ctypes.c_float)]
+        "k_b", "k_t", "max_ctx", "kv_dtype", "out_dtype")] + [("softmax_scale", ctypes.c_float),
+                                                               ("block_agg", ctypes.c_int32)]
 
     def __repr__(self):
         return "TlsShape(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -77,20 +78,22 @@ for _name, (_args, _ret) in _sigs.items():
 
 
 def make_shape(batch, n_q_heads, n_kv_heads, d_qk, d_v, block_size, n_label, k_b, k_t, max_ctx, kv_dtype,
-               out_dtype=TLS_F32, v_is_k_prefix=False, softmax_scale: Optional[float] = None) -> TlsShape:
+               out_dtype=TLS_F32, v_is_k_prefix=False, softmax_scale: Optional[float] = None,
+               block_agg: int = 0) -> TlsShape:
     s = TlsShape()
     s.batch, s.n_q_heads, s.n_kv_heads = batch, n_q_heads, n_kv_heads
     s.d_qk, s.d_v, s.v_is_k_prefix = d_qk, d_v, int(bool(v_is_k_prefix))
     s.block_size, s.n_label, s.k_b, s.k_t, s.max_ctx = block_size, n_label, k_b, k_t, max_ctx
     s.kv_dtype, s.out_dtype = kv_dtype, out_dtype
     s.softmax_scale = (1.0 / math.sqrt(d_qk)) if softmax_scale is None else softmax_scale
+    s.block_agg = int(block_agg)
     return s
 
 
 def shape_from_workload(w, out_dtype=TLS_F32, **over) -> TlsShape:
     kw = dict(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, d_qk=w.d_qk, d_v=w.d_v,
               block_size=w.block_size, n_label=w.n_label, k_b=w.k_b, k_t=w.k_t, max_ctx=w.ctx, kv_dtype=w.dtype,
-              out_dtype=out_dtype, v_is_k_prefix=w.v_is_k_prefix)
+              out_dtype=out_dtype, v_is_k_prefix=w.v_is_k_prefix, block_agg=getattr(w, "block_agg", 0))
     kw.update(over)
     return make_shape(**kw)
 
