@@ -244,7 +244,7 @@ def gpu_arm(args, rank, world, local_rank):
     # ---- timed region: K steps.  Kernels within and across stages are chained by
     # programmatic dependent launch; per-stage CUDA events (which break that
     # overlap at the stage boundaries) are recorded on every SAMPLE-th step only.
-    SAMPLE = 8
+    SAMPLE = 32
     evs = {i: [torch.cuda.Event(enable_timing=True) for _ in range(3)] for i in range(0, args.steps, SAMPLE)}
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
