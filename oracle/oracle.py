@@ -27,7 +27,8 @@ _lib = None
 class OraShape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "batch", "n_q_heads", "n_kv_heads", "d_qk", "d_v", "v_is_k_prefix",
-        "block_size", "n_label", "k_b", "k_t", "max_ctx", "dtype", "block_agg")] + [("softmax_scale", ctypes.c_double)]
+        "block_size", "n_label", "k_b", "k_t", "max_ctx", "dtype", "block_agg", "slab_bits")] + [
+            ("softmax_scale", ctypes.c_double)]
 
 
 def build(force: bool = False) -> str:
@@ -57,8 +58,9 @@ def lib():
         L.ora_select_tokens.argtypes = [S, P, P, i, P]
         L.ora_attention.argtypes = [S, P, P, P, P, P, P]
         L.ora_decode_step.argtypes = [S, P, P, P, P, P, P, i, P, P, P, P]
+        L.ora_quantize_labels.argtypes = [S, P, P, P, P, P]
         for f in ("ora_build_meta", "ora_block_scores", "ora_select_blocks", "ora_token_scores",
-                  "ora_select_tokens", "ora_attention", "ora_decode_step"):
+                  "ora_select_tokens", "ora_attention", "ora_decode_step", "ora_quantize_labels"):
             getattr(L, f).restype = None
         _lib = L
     return _lib
@@ -74,6 +76,7 @@ def shape_of(w, k_b: Optional[int] = None, k_t: Optional[int] = None, softmax_sc
     s.k_t = w.k_t if k_t is None else k_t
     s.max_ctx, s.dtype = w.ctx, w.dtype
     s.block_agg = int(getattr(w, "block_agg", 0))
+    s.slab_bits = int(getattr(w, "slab_bits", 0))
     s.softmax_scale = (1.0 / math.sqrt(w.d_qk)) if softmax_scale is None else softmax_scale
     return s
 
@@ -155,6 +158,16 @@ def decode_step(s, q, K, V, meta, seq_lens, label_idx, decide_f32: bool = False,
                           _p(np.ascontiguousarray(label_idx, np.int32)), int(decide_f32),
                           _p(bidx), _p(tidx), _p(out), _p(lse))
     return bidx, tidx, out, lse
+
+
+def quantize_labels(s, K, seq_lens, label_idx):
+    """The int8 label codes and their per-channel scales (the quantised slab
+    reading); returns (codes [B][H_kv][max_ctx][r] int8, scales [B][H_kv][r] fp32)."""
+    codes = np.empty((s.batch, s.n_kv_heads, s.max_ctx, s.n_label), np.int8)
+    scales = np.empty((s.batch, s.n_kv_heads, s.n_label), np.float32)
+    lib().ora_quantize_labels(ctypes.byref(s), _p(K), _p(np.ascontiguousarray(seq_lens, np.int32)),
+                              _p(np.ascontiguousarray(label_idx, np.int32)), _p(codes), _p(scales))
+    return codes, scales
 
 
 def label_slab(s, K, label_idx) -> np.ndarray:

@@ -35,6 +35,7 @@ typedef struct {
   int batch, n_q_heads, n_kv_heads, d_qk, d_v, v_is_k_prefix;
   int block_size, n_label, k_b, k_t, max_ctx, dtype; /* dtype 0: fp32, 1: bf16 bits */
   int block_agg;                                      /* 0: sum of the heads' bounds, 1: their max */
+  int slab_bits;                                      /* 0: exact label channels, 8: int8 codes */
   double softmax_scale;
 } ora_shape;
 
@@ -179,10 +180,20 @@ void ora_select_blocks(const ora_shape *s, const double *score, const int32_t *s
  * invalid when that block id is -1 or the token is at or beyond seq_len.
  * cand_score / cand_tok: [B][H_kv][k_b * bs]; invalid -> -inf / -1.
  * The scores are computed from K itself (not from any copied slab). */
+void ora_quantize_labels(const ora_shape *s, const void *K, const int32_t *seq_lens, const int32_t *label_idx,
+                         int8_t *codes, float *scales);
+
 void ora_token_scores(const ora_shape *s, const void *q, const void *K, const int32_t *label_idx,
                       const int32_t *block_idx, const int32_t *seq_lens, double *cand_score, int32_t *cand_tok) {
   const int d = s->d_qk, G = s->n_q_heads / s->n_kv_heads, bs = s->block_size;
   const int C = s->k_b * bs;
+  int8_t *codes = NULL;
+  float *scales = NULL;
+  if (s->slab_bits == 8) {  /* the quantised variant: K[t, L_c] is replaced by scale_c * code */
+    codes = (int8_t *)malloc((size_t)s->batch * s->n_kv_heads * s->max_ctx * s->n_label);
+    scales = (float *)malloc(sizeof(float) * (size_t)s->batch * s->n_kv_heads * s->n_label);
+    ora_quantize_labels(s, K, seq_lens, label_idx, codes, scales);
+  }
   for (int b = 0; b < s->batch; ++b)
     for (int g = 0; g < s->n_kv_heads; ++g) {
       const size_t bg = (size_t)b * s->n_kv_heads + g;
@@ -197,12 +208,60 @@ void ora_token_scores(const ora_shape *s, const void *q, const void *K, const in
           const int h = g * G + hh;
           for (int c = 0; c < s->n_label; ++c) {
             const int ch = label_idx[c];
-            acc += ora_in(q, s->dtype, ((size_t)b * s->n_q_heads + h) * d + ch) *
-                   ora_in(K, s->dtype, (bg * s->max_ctx + t) * d + ch);
+            if (ch < 0 || ch >= d) continue;
+            const double kv = codes ? (double)scales[bg * s->n_label + c] *
+                                          (double)codes[(bg * s->max_ctx + t) * s->n_label + c]
+                                    : ora_in(K, s->dtype, (bg * s->max_ctx + t) * d + ch);
+            acc += ora_in(q, s->dtype, ((size_t)b * s->n_q_heads + h) * d + ch) * kv;
           }
         }
         *os = acc;
         *ot = t;
+      }
+    }
+  free(codes);
+  free(scales);
+}
+
+/* ---- the quantised label slab (variant) -----------------------------------
+ * gist.science (de) section 2.A "Stufe 2": the token stage reads the label
+ * channels "durch Quantisierung und Kanalauswahl" (through quantisation and
+ * channel choice).  Reading: per sequence, KV head and label channel c, a
+ * symmetric scale = max |K[t, L_c]| over the valid tokens / 127 and codes
+ * round-half-even(K / scale) clamped to [-127, 127] (scale 0: codes 0).  The
+ * scale and the codes are integers decided from fp32 values, so they are
+ * computed in fp32 here (IEEE division, rint) as any implementation that
+ * shares the reading must; the token score then uses scale * code in fp64.
+ * codes: [B][H_kv][max_ctx][r] (rows >= seq_len: 0); scales: [B][H_kv][r]. */
+void ora_quantize_labels(const ora_shape *s, const void *K, const int32_t *seq_lens, const int32_t *label_idx,
+                         int8_t *codes, float *scales) {
+  const int d = s->d_qk, r = s->n_label;
+  for (int b = 0; b < s->batch; ++b)
+    for (int g = 0; g < s->n_kv_heads; ++g) {
+      const size_t bg = (size_t)b * s->n_kv_heads + g;
+      const int L = seq_lens[b] < 0 ? 0 : (seq_lens[b] > s->max_ctx ? s->max_ctx : seq_lens[b]);
+      for (int c = 0; c < r; ++c) {
+        const int ch = label_idx[c];
+        float maxabs = 0.0f;
+        if (ch >= 0 && ch < d)
+          for (int t = 0; t < L; ++t) {
+            const size_t ki = (bg * s->max_ctx + t) * d + ch;
+            const float v = (float)ora_in(K, s->dtype, ki);
+            const float a = v < 0.0f ? -v : v;
+            if (a > maxabs) maxabs = a;
+          }
+        const float scale = maxabs / 127.0f;
+        scales[bg * r + c] = scale;
+        for (int t = 0; t < s->max_ctx; ++t) {
+          int code = 0;
+          if (t < L && scale > 0.0f && ch >= 0 && ch < d) {
+            const size_t ki = (bg * s->max_ctx + t) * d + ch;
+            const float v = (float)ora_in(K, s->dtype, ki);
+            const float qv = rintf(v / scale);
+            code = qv > 127.0f ? 127 : (qv < -127.0f ? -127 : (int)qv);
+          }
+          codes[(bg * s->max_ctx + t) * r + c] = (int8_t)code;
+        }
       }
     }
 }

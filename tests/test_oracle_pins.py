@@ -475,3 +475,75 @@ def test_planted_mistake_is_caught(name):
     finally:
         O._lib = saved
         shutil.rmtree(tmp, ignore_errors=True)
+
+
+# --------------------------------------------------------------------------- quantised label slab
+@pytest.mark.parametrize("dtype", [W.F32, W.BF16])
+def test_quantized_label_codes_properties(dtype):
+    """Codes are integers in [-127, 127] (0 past seq_len), scale * code is within
+    scale / 2 of the stored value, the largest |K| of a channel maps to +-127,
+    and an all-zero channel has scale 0 and codes 0."""
+    sh = Sh(batch=2, n_q_heads=4, n_kv_heads=2, ctx=64, block_size=8, d_qk=16, n_label=8, dtype=dtype, slab_bits=8)
+    q, K, V, sl = rand_inputs(sh, 5, dtype=dtype, seq_lens=[64, 37])
+    label = np.array([0, 3, 5, 6, 9, 11, 12, 15], np.int32)
+    if dtype == W.F32:
+        K[:, :, :, 6] = 0.0  # label channel 3: all zero
+    else:
+        K[:, :, :, 6] = 0
+    s = O.shape_of(sh)
+    codes, scales = O.quantize_labels(s, K, sl, label)
+    Kf = f64(K, dtype)
+    for b in range(sh.batch):
+        L = int(sl[b])
+        assert (codes[b, :, L:] == 0).all()
+        for g in range(sh.n_kv_heads):
+            for c, ch in enumerate(label):
+                col = Kf[b, g, :L, ch]
+                sc = float(scales[b, g, c])
+                if np.abs(col).max() == 0:
+                    assert sc == 0 and (codes[b, g, :L, c] == 0).all()
+                    continue
+                cd = codes[b, g, :L, c].astype(np.float64)
+                assert np.abs(cd).max() == 127 and abs(cd[np.abs(col).argmax()]) == 127
+                assert (np.abs(sc * cd - col) <= 0.5 * sc * (1 + 1e-6) + 1e-30).all()
+
+
+def test_quantized_token_scores_within_the_quantization_bound():
+    sh = Sh(batch=2, n_q_heads=8, n_kv_heads=2, ctx=96, block_size=8, d_qk=16, n_label=8, k_b=6, k_t=20)
+    q, K, V, sl = rand_inputs(sh, 9, seq_lens=[96, 61])
+    label = np.array([1, 2, 4, 7, 8, 10, 13, 14], np.int32)
+    s = O.shape_of(sh)
+    s8 = O.shape_of(Sh(**{**sh.__dict__, "slab_bits": 8}))
+    bidx = O.select_blocks(s, O.block_scores(s, q, O.build_meta(s, K, sl), sl), sl)
+    exact, tok = O.token_scores(s, q, K, label, bidx, sl)
+    quant, tok8 = O.token_scores(s8, q, K, label, bidx, sl)
+    np.testing.assert_array_equal(tok, tok8)
+    _, scales = O.quantize_labels(s8, K, sl, label)
+    qf = f64(q, W.F32).reshape(sh.batch, sh.n_kv_heads, 4, sh.d_qk)[..., label]  # [B][H][G][r]
+    bound = (np.abs(qf).sum(axis=2) * scales * 0.5).sum(axis=-1)  # [B][H]
+    ok = tok >= 0
+    diff = np.where(ok, np.abs(quant - exact), 0)
+    assert (diff <= bound[:, :, None] * (1 + 1e-6)).all()
+    assert diff.max() > 0  # the variant does change the scores
+
+
+def test_quantized_token_scores_exact_on_a_power_of_two_grid():
+    """K values m * 2^-3 with integer |m| <= 127 and 127 reached in every label
+    channel: scale = 2^-3 exactly, codes = m, scores equal the exact ones."""
+    sh = Sh(batch=1, n_q_heads=2, n_kv_heads=1, ctx=32, block_size=8, d_qk=8, n_label=4, k_b=4, k_t=10)
+    rng = np.random.default_rng(3)
+    m = rng.integers(-127, 128, size=(1, 1, 32, 8)).astype(np.float32)
+    m[0, 0, 5, :] = 127.0
+    K = (m / 8.0).astype(np.float32)
+    q = rng.standard_normal((1, 2, 8)).astype(np.float32)
+    sl = np.array([32], np.int32)
+    label = np.array([0, 2, 5, 7], np.int32)
+    s = O.shape_of(sh)
+    s8 = O.shape_of(Sh(**{**sh.__dict__, "slab_bits": 8}))
+    codes, scales = O.quantize_labels(s8, K, sl, label)
+    assert (scales == np.float32(0.125)).all()
+    np.testing.assert_array_equal(codes[0, 0, :, :], m[0, 0][:, label].astype(np.int8))
+    bidx = np.array([[[0, 1, 2, 3]]], np.int32)
+    exact, _ = O.token_scores(s, q, K, label, bidx, sl)
+    quant, _ = O.token_scores(s8, q, K, label, bidx, sl)
+    np.testing.assert_array_equal(quant, exact)

@@ -58,6 +58,7 @@ class Workload:
     seed: int
     steps: int = 1          # decode steps (> 1 only for the AR(1) query stream)
     block_agg: int = 0      # block score over the group's heads: 0 sum (the method), 1 max (variant)
+    slab_bits: int = 0      # label slab: 0 the K dtype, 8 int8 codes with per-channel scales (variant)
     ar_rho: float = 0.0     # q_t = rho q_{t-1} + sqrt(1 - rho^2) N(0, I)
 
     @property
