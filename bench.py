@@ -47,7 +47,8 @@ def algorithmic_bytes(w) -> dict:
     vrow = 0 if w.v_is_k_prefix else w.d_v
     parts = {
         "block_summary": G * w.n_blocks * 2 * w.d_qk * e,
-        "label_slab": G * w.k_b * w.block_size * w.n_label * e,
+        "label_slab": (G * w.k_b * w.block_size * w.n_label * e if getattr(w, "slab_bits", 0) != 8
+                       else G * w.k_b * w.block_size * w.n_label + G * w.n_label * 4),  # int8 codes + scales
         "gathered_kv": G * w.k_t * (w.d_qk + vrow) * e,
         "q": w.batch * w.n_q_heads * w.d_qk * e,
         "out_lse": w.batch * w.n_q_heads * (w.d_v * 4 + 4),
@@ -183,7 +184,10 @@ class Layer:
         self.q = q
         edt = torch.int16 if w.dtype == 1 else torch.float32
         self.meta = torch.empty((w.batch, w.n_kv_heads, w.n_blocks, 2, w.d_qk), dtype=edt, device=dev)
-        self.slab = torch.empty((w.batch, w.n_kv_heads, w.ctx, w.n_label), dtype=edt, device=dev)
+        if shape.slab_bits == 8:
+            self.slab = torch.empty(T.tls_slab_bytes(shape), dtype=torch.uint8, device=dev)
+        else:
+            self.slab = torch.empty((w.batch, w.n_kv_heads, w.ctx, w.n_label), dtype=edt, device=dev)
         T.tls_build_block_meta(shape, self.K, seq_lens, label, self.meta, self.slab)
 
 
@@ -200,7 +204,7 @@ def gpu_arm(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    base = W.WORKLOADS[args.workload]
+    base = W.WORKLOADS[args.workload].with_(slab_bits=args.slab_bits)
     w = rank_workload(base, rank)
     shape = T.shape_from_workload(w)
     inp = W.make_decode_inputs(w)
@@ -352,7 +356,7 @@ def gpu_arm(args, rank, world, local_rank):
         "config": {
             "workload": args.workload, "batch": w.batch, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
             "d_qk": w.d_qk, "d_v": w.d_v, "ctx": w.ctx, "block_size": w.block_size, "k_b": w.k_b, "k_t": w.k_t,
-            "n_label": w.n_label, "out_dtype": "f32",
+            "n_label": w.n_label, "out_dtype": "f32", "label_slab": "int8" if w.slab_bits == 8 else "kv dtype",
             "l2": f"inputs larger than L2: {N_LAYERS} layer copies rotated, {N_LAYERS * ab['total'] / 1e6:.0f} MB "
                   f"of algorithmic bytes per rotation (L2 126 MB)",
             "algorithmic_bytes_per_step": ab["total"],
@@ -587,6 +591,8 @@ def main():
                     help="time full-attention decode (all tokens selected) of the workload, for context")
     ap.add_argument("--offload", action="store_true",
                     help="time the offload engine on the streaming workload instead (one JSON line of its own)")
+    ap.add_argument("--slab-bits", type=int, default=0, choices=[0, 8],
+                    help="label slab storage: 0 = the K dtype (the method), 8 = int8 codes + per-channel scales")
     ap.add_argument("--layers", type=int, default=N_LAYERS_DEFAULT,
                     help="layer copies rotated through (4 keeps the per-rotation working set above L2)")
     args = ap.parse_args()

@@ -84,6 +84,8 @@ typedef struct tls_shape {
   float softmax_scale;   /* tau; <= 0 selects 1/sqrt(d_qk)                               */
   int32_t block_agg;     /* block score over the group's heads: 0 = sum of the heads'
                           * bounds (the method), 1 = their maximum (a variant; GQA only)  */
+  int32_t slab_bits;     /* label slab: 0 = the K dtype; 8 = int8 codes with one fp32 scale
+                          * per (sequence, KV head, label channel) (bf16 K, r in {16,32,64}) */
 } tls_shape;
 
 /* Supported shapes (others return TLS_ERR_UNSUPPORTED):
@@ -108,6 +110,12 @@ TLS_API const char *tls_last_error(void);
  * NULL.  Returns 0 for an invalid shape (see tls_last_error). */
 TLS_API size_t tls_workspace_size(const tls_shape *s);
 
+/* Bytes of the label slab buffer for this shape: B*H_kv*max_ctx*r elements of
+ * the K dtype (slab_bits 0), or, for slab_bits 8, B*H_kv*max_ctx*r int8 codes
+ * followed (at the next multiple of 256 bytes) by B*H_kv*r fp32 scales.
+ * Returns 0 for an invalid shape. */
+TLS_API size_t tls_slab_bytes(const tls_shape *s);
+
 /* Set-up: block summary and label-channel slab of a KV cache.
  * gist.science (de) section 2.A "Stufe 1": blocks are summarised by the
  * per-channel maximum and minimum of their keys; (es) section 2.A.2: token
@@ -119,7 +127,11 @@ TLS_API size_t tls_workspace_size(const tls_shape *s);
  *              over the block's tokens t < seq_len (a partial last block uses its
  *              valid part; blocks with no valid token are left untouched)
  *   slab_out   device [B][H_kv][max_ctx][n_label]: slab[.., t, c] = K[.., t, label_idx[c]]
- *              for t < seq_len (other rows untouched); may be NULL to skip. */
+ *              for t < seq_len (other rows untouched); may be NULL to skip.
+ *              slab_bits 8 (the quantised variant): tls_slab_bytes(s) bytes holding
+ *              the codes round-half-even(K / scale) clamped to [-127, 127] (rows
+ *              >= seq_len: 0) and the scales max|K[.., t < seq_len, L_c]| / 127,
+ *              both decided in fp32 (the max comes from the block summary). */
 TLS_API tls_status tls_build_block_meta(const tls_shape *s, const void *K, const int32_t *seq_lens,
                                 const int32_t *label_idx, void *meta_out, void *slab_out, void *stream);
 

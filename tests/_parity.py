@@ -72,7 +72,10 @@ class GpuInputs:
         edt = torch.int16 if w.dtype == W.BF16 else torch.float32
         B, H, nb, d = w.batch, w.n_kv_heads, w.n_blocks, w.d_qk
         self.meta = torch.zeros((B, H, nb, 2, d), dtype=edt, device="cuda")
-        self.slab = torch.zeros((B, H, w.ctx, w.n_label), dtype=edt, device="cuda")
+        if getattr(w, "slab_bits", 0) == 8:  # int8 codes + fp32 scales in one buffer
+            self.slab = torch.zeros(T.tls_slab_bytes(self.shape), dtype=torch.uint8, device="cuda")
+        else:
+            self.slab = torch.zeros((B, H, w.ctx, w.n_label), dtype=edt, device="cuda")
         T.tls_build_block_meta(self.shape, self.K, self.seq_lens, self.label, self.meta, self.slab)
         self.ws = torch.zeros(T.tls_workspace_size(self.shape), dtype=torch.uint8, device="cuda")
 
@@ -123,6 +126,9 @@ def check_meta(w, inp, gpu: GpuInputs, orc: OracleRun):
     for b in range(w.batch):
         nb = -(-int(inp.seq_lens[b]) // w.block_size)
         np.testing.assert_array_equal(gm[b, :, :nb], orc.meta[b, :, :nb])
+    if getattr(w, "slab_bits", 0) == 8:
+        check_slab_q8(w, inp, gpu)
+        return
     # the slab is a copy of stored values: compare the stored bits
     gs = gpu.slab.cpu().numpy()
     gs = gs.view(np.uint16) if w.dtype == W.BF16 else gs.view(np.uint32)
@@ -130,6 +136,27 @@ def check_meta(w, inp, gpu: GpuInputs, orc: OracleRun):
     for b in range(w.batch):
         L = int(inp.seq_lens[b])
         np.testing.assert_array_equal(gs[b, :, :L], Kr[b, :, :L][..., inp.label_idx])
+
+
+def slab_q8_views(w, slab: np.ndarray):
+    """(codes [B][H][ctx][r] int8, scales [B][H][r] fp32) of an int8 slab buffer:
+    the codes, then the scales at the next multiple of 256 bytes."""
+    n = w.batch * w.n_kv_heads * w.ctx * w.n_label
+    off = -(-n // 256) * 256
+    codes = slab[:n].view(np.int8).reshape(w.batch, w.n_kv_heads, w.ctx, w.n_label)
+    scales = slab[off:off + 4 * w.batch * w.n_kv_heads * w.n_label].view(np.float32)
+    return codes, scales.reshape(w.batch, w.n_kv_heads, w.n_label)
+
+
+def check_slab_q8(w, inp, gpu: GpuInputs):
+    """Codes and scales are integers / fp32 values decided in fp32 on both
+    sides: bit-exact on the valid rows."""
+    codes, scales = slab_q8_views(w, gpu.slab.cpu().numpy())
+    oc, osc = O.quantize_labels(O.shape_of(w), inp.K, inp.seq_lens, inp.label_idx)
+    np.testing.assert_array_equal(scales.view(np.uint32), osc.view(np.uint32))
+    for b in range(w.batch):
+        L = int(inp.seq_lens[b])
+        np.testing.assert_array_equal(codes[b, :, :L], oc[b, :, :L])
 
 
 def block_score_bound(w, inp, orc: OracleRun) -> np.ndarray:
@@ -144,7 +171,9 @@ def block_score_bound(w, inp, orc: OracleRun) -> np.ndarray:
 
 def token_score_bound(w, inp, orc: OracleRun, block_idx: np.ndarray) -> np.ndarray:
     """fp32 rounding bound of the kernel's token score: Qbar_L = sum of G heads,
-    then an r-term dot; each term bounded by |q_{h,c}| |K[t,c]|."""
+    then an r-term dot; each term bounded by |q_{h,c}| |K[t,c]| (int8 slab:
+    |q_{h,c}| |scale_c code|, one more rounding for the folded scale)."""
+    q8 = O.quantize_labels(O.shape_of(w), inp.K, inp.seq_lens, inp.label_idx) if getattr(w, "slab_bits", 0) == 8 else None
     q = W.to_f64(inp.q, w.dtype).reshape(w.batch, w.n_kv_heads, w.group, w.d_qk)[..., inp.label_idx]
     C = w.k_b * w.block_size
     out = np.zeros((w.batch, w.n_kv_heads, C))
@@ -154,10 +183,13 @@ def token_score_bound(w, inp, orc: OracleRun, block_idx: np.ndarray) -> np.ndarr
             blk = block_idx[b, g][j // w.block_size]
             t = blk * w.block_size + j % w.block_size
             ok = (blk >= 0) & (t < inp.seq_lens[b])
-            rows = inp.K[b, g][np.where(ok, t, 0)][:, inp.label_idx]
-            kk = np.abs(W.to_f64(rows, w.dtype))
+            if q8 is not None:  # |scale_c * code| in place of |K[t, L_c]|
+                kk = np.abs(q8[0][b, g][np.where(ok, t, 0)].astype(np.float64) * q8[1][b, g].astype(np.float64))
+            else:
+                rows = inp.K[b, g][np.where(ok, t, 0)][:, inp.label_idx]
+                kk = np.abs(W.to_f64(rows, w.dtype))
             out[b, g] = np.where(ok, kk @ np.abs(q[b, g]).sum(axis=0), 0.0)
-    return 2.0 * (w.n_label + w.group + 2) * U32 * out
+    return 2.0 * (w.n_label + w.group + 2 + (q8 is not None)) * U32 * out
 
 
 def check_scores(gpu_scores: np.ndarray, ora_scores: np.ndarray, bound: np.ndarray, what: str):

@@ -125,6 +125,30 @@ def test_block_aggregation_field_is_checked(T):
     assert call_block(T, mla) == T.TLS_ERR_UNSUPPORTED
 
 
+def test_int8_slab_field_and_size(T):
+    s = good_shape(T)
+    n0 = T.tls_slab_bytes(s)
+    assert n0 == s.batch * s.n_kv_heads * s.max_ctx * s.n_label * (2 if s.kv_dtype == T.TLS_BF16 else 4)
+    s.slab_bits = 8
+    if s.kv_dtype == T.TLS_BF16 and s.n_label >= 16:
+        codes = s.batch * s.n_kv_heads * s.max_ctx * s.n_label
+        assert T.tls_slab_bytes(s) == -(-codes // 256) * 256 + 4 * s.batch * s.n_kv_heads * s.n_label
+    s.slab_bits = 4
+    assert call_block(T, s) == T.TLS_ERR_INVALID_ARG and "slab_bits" in T.tls_last_error()
+    f32 = good_shape(T, kv_dtype=T.TLS_F32, n_label=16)
+    f32.slab_bits = 8
+    assert call_block(T, f32) == T.TLS_ERR_UNSUPPORTED and "int8" in T.tls_last_error()
+    r8 = good_shape(T, kv_dtype=T.TLS_BF16, n_label=8)
+    r8.slab_bits = 8
+    assert call_block(T, r8) == T.TLS_ERR_UNSUPPORTED
+    with pytest.raises(T.TlsError):
+        T.tls_slab_bytes(r8)
+    q8 = good_shape(T, kv_dtype=T.TLS_BF16, n_label=16)
+    q8.slab_bits = 8
+    st = T._lib.tls_append_tokens(ctypes.byref(q8), 256, 256, 256, 4, 256, 256, 256, None)
+    assert st == T.TLS_ERR_UNSUPPORTED and "int8" in T.tls_last_error()
+
+
 def test_select_step_checks_before_launch(T):
     s = good_shape(T)
     st = T._lib.tls_select_step(ctypes.byref(s), 256, 256, None, 256, 256, 256, 256, None, None, None)

@@ -158,3 +158,39 @@ def test_alternative_attention_kernels_parity(impl):
     env = dict(os.environ, TLS_ATTN_IMPL=impl)
     r = subprocess.run([sys.executable, "-c", code], env=env, cwd=root, capture_output=True, text=True, timeout=900)
     assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout[-2000:] + r.stderr[-4000:]
+
+
+SLAB_Q8 = {
+    # the int8 label slab: codes and scales bit-exact, token scores and
+    # selections against the oracle's quantised reading
+    "q8_r16_ragged": (W.WORKLOADS["gqa48k_bf16"].with_(batch=2, ctx=4096, k_b=24, k_t=300, slab_bits=8),
+                      [4096, 3001]),
+    "q8_r32_g8": (W.WORKLOADS["gqa48k_bf16"].with_(n_q_heads=64, ctx=2048, k_b=16, k_t=257, n_label=32,
+                                                   slab_bits=8), None),
+    "q8_r64_d64_empty": (W.WORKLOADS["gqa48k_bf16"].with_(batch=4, n_q_heads=16, d_qk=64, d_v=64, ctx=512, k_b=4,
+                                                          k_t=40, n_label=64, slab_bits=8), [0, 1, 31, 512]),
+    "q8_mla_small": (W.WORKLOADS["mla64k_b4_bf16"].with_(batch=2, ctx=4096, k_b=16, k_t=300, n_needles=4,
+                                                         slab_bits=8), [4096, 3000]),
+    "q8_full_gqa96k_b8": (W.WORKLOADS["gqa96k_b8_bf16"].with_(slab_bits=8), None),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SLAB_Q8))
+def test_int8_label_slab_parity(name):
+    w, sl = SLAB_Q8[name]
+    res = P().full_stage_parity(w, seq_lens=sl, name=name)
+    assert res["token_swaps"] <= max(1, res["groups"] // 8)
+
+
+def test_int8_label_slab_select_step_equals_separate_calls():
+    from tests import _parity as PP
+    from two_level_sparse_quest_b200 import tls as T
+
+    w = W.WORKLOADS["gqa48k_bf16"].with_(batch=2, ctx=4096, k_b=24, k_t=300, slab_bits=8)
+    g = PP.GpuInputs(w, W.make_decode_inputs(w, seq_lens=[4096, 2222]))
+    bidx, _ = g.block_stage()
+    tidx, _ = g.token_stage(bidx)
+    fb, ft = torch.full_like(bidx, -7), torch.full_like(tidx, -7)
+    T.tls_select_step(g.shape, g.q, g.meta, g.slab, g.label, g.seq_lens, fb, ft)
+    torch.cuda.synchronize()
+    assert torch.equal(fb, bidx) and torch.equal(ft, tidx)

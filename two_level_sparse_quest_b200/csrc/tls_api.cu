@@ -92,7 +92,26 @@ tls_status check_shape(const tls_shape *s) {
                         : (s->n_label == 4 || s->n_label == 8 || s->n_label == 16 || s->n_label == 32);
   if (!r_ok) return fail(TLS_ERR_UNSUPPORTED, "n_label %d unsupported for this dtype", s->n_label);
   if (s->n_label > s->d_qk) return fail(TLS_ERR_INVALID_ARG, "n_label > d_qk");
+  if (s->slab_bits != 0 && s->slab_bits != 8) return fail(TLS_ERR_INVALID_ARG, "slab_bits %d", s->slab_bits);
+  if (s->slab_bits == 8 && (s->kv_dtype != TLS_BF16 || s->n_label < 16))
+    return fail(TLS_ERR_UNSUPPORTED, "the int8 label slab needs bf16 keys and n_label in {16, 32, 64}");
   return TLS_OK;
+}
+
+// Label slab layout: the slab of the K dtype, or int8 codes followed by the
+// fp32 scales at the next multiple of 256 bytes.
+size_t slab_codes_bytes(const tls_shape *s) {
+  const size_t rows = static_cast<size_t>(s->batch) * s->n_kv_heads * s->max_ctx * s->n_label;
+  return s->slab_bits == 8 ? rows : rows * (s->kv_dtype == TLS_BF16 ? 2 : 4);
+}
+size_t slab_scales_offset(const tls_shape *s) { return (slab_codes_bytes(s) + 255) / 256 * 256; }
+size_t slab_total_bytes(const tls_shape *s) {
+  if (s->slab_bits != 8) return slab_codes_bytes(s);
+  return slab_scales_offset(s) + sizeof(float) * static_cast<size_t>(s->batch) * s->n_kv_heads * s->n_label;
+}
+const float *slab_scales(const tls_shape *s, const void *slab) {
+  if (s->slab_bits != 8) return nullptr;
+  return reinterpret_cast<const float *>(static_cast<const char *>(slab) + slab_scales_offset(s));
 }
 
 #define CHECK_PTR(p, a)                                                                          \
@@ -195,6 +214,11 @@ size_t tls_workspace_size(const tls_shape *s) {
   return w.total;
 }
 
+size_t tls_slab_bytes(const tls_shape *s) {
+  if (check_shape(s) != TLS_OK) return 0;
+  return slab_total_bytes(s);
+}
+
 tls_status tls_build_block_meta(const tls_shape *s, const void *K, const int32_t *seq_lens, const int32_t *label_idx,
                                 void *meta_out, void *slab_out, void *stream) {
   tls_status st = check_shape(s);
@@ -212,6 +236,13 @@ tls_status tls_build_block_meta(const tls_shape *s, const void *K, const int32_t
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   st = cuda_status(tls::launch_build_meta(a, cs), "build_meta launch");
   if (st != TLS_OK || !slab_out) return st;
+  if (s->slab_bits == 8) {
+    // the scales come from the block summary just written (stream order)
+    float *scales = const_cast<float *>(slab_scales(s, slab_out));
+    st = cuda_status(tls::launch_label_scales(a, scales, cs), "label_scales launch");
+    if (st != TLS_OK) return st;
+    return cuda_status(tls::launch_build_slab_q8(a, scales, cs), "build_slab_q8 launch");
+  }
   return cuda_status(tls::launch_build_slab(a, cs), "build_slab launch");
 }
 
@@ -227,6 +258,8 @@ tls_status tls_append_tokens(const tls_shape *s, const void *K, const int32_t *o
   CHECK_PTR(new_lens, 4);
   CHECK_PTR(meta, 16);
   if (slab) {
+    if (s->slab_bits == 8)  // an append can move a channel's scale and so every code of the group
+      return fail(TLS_ERR_UNSUPPORTED, "tls_append_tokens does not update an int8 label slab; rebuild it");
     CHECK_PTR(label_idx, 4);
     CHECK_PTR(slab, 4);
   }
@@ -270,7 +303,7 @@ tls_status tls_token_score_topk(const tls_shape *s, const void *q, const void *s
   if (token_score_out && !aligned(token_score_out, 4)) return fail(TLS_ERR_INVALID_ARG, "token_score_out misaligned");
   tls::TokenArgs a{q, slab, label_idx, block_idx, seq_lens, token_idx_out, token_score_out, s->batch, s->n_q_heads,
                    s->n_kv_heads, s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->n_label, s->k_b, s->k_t,
-                   s->kv_dtype, tls::device_error_word()};
+                   s->kv_dtype, tls::device_error_word(), slab_scales(s, slab)};
   (void)ws;  // the selection keeps its keys in on-chip memory: no workspace
   (void)ws_bytes;
   return cuda_status(tls::launch_token_select(a, static_cast<cudaStream_t>(stream)), "token_select launch");
@@ -296,7 +329,7 @@ tls_status tls_select_step(const tls_shape *s, const void *q, const void *meta, 
                         s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->k_b, s->kv_dtype, err, s->block_agg};
   tls::TokenArgs t{q, slab, label_idx, block_idx_out, seq_lens, token_idx_out, token_score_out, s->batch, s->n_q_heads,
                    s->n_kv_heads, s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->n_label, s->k_b, s->k_t,
-                   s->kv_dtype, err};
+                   s->kv_dtype, err, slab_scales(s, slab)};
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   if (s->block_agg == 1) {  // the max-over-heads variant runs as the two separate launches
     st = cuda_status(tls::launch_block_select(a, cs), "block_select launch");

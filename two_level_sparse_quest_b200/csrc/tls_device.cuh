@@ -22,6 +22,11 @@ struct BF16 {
   static constexpr int kBytes = 2;
   static constexpr int kEPC = 8;
 };
+struct I8 {  // int8 codes of the quantised label slab
+  using storage = int8_t;
+  static constexpr int kBytes = 1;
+  static constexpr int kEPC = 16;
+};
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
@@ -42,6 +47,14 @@ __device__ __forceinline__ void chunk_to_f32<BF16>(const uint4 &c, float *f) {
   f[2] = bf16_lo(c.y); f[3] = bf16_hi(c.y);
   f[4] = bf16_lo(c.z); f[5] = bf16_hi(c.z);
   f[6] = bf16_lo(c.w); f[7] = bf16_hi(c.w);
+}
+template <>
+__device__ __forceinline__ void chunk_to_f32<I8>(const uint4 &c, float *f) {
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) f[4 * i + k] = static_cast<float>(static_cast<int32_t>(w[i] << (24 - 8 * k)) >> 24);
 }
 
 template <typename E>

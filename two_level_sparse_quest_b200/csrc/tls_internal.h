@@ -62,6 +62,10 @@ struct MetaArgs {
 };
 cudaError_t launch_build_meta(const MetaArgs &a, cudaStream_t st);
 cudaError_t launch_build_slab(const MetaArgs &a, cudaStream_t st);
+// int8 label slab (bf16 keys): scales[group][c] = max |K[t < seq, L_c]| / 127
+// from the block summary a.meta, then the codes into a.slab.
+cudaError_t launch_label_scales(const MetaArgs &a, float *scales, cudaStream_t st);
+cudaError_t launch_build_slab_q8(const MetaArgs &a, const float *scales, cudaStream_t st);
 // Incremental update after appending tokens [old_lens[b], new_lens[b]) to K:
 // rebuilds the summaries of the blocks those rows fall in and their slab rows.
 struct AppendArgs {
@@ -95,6 +99,7 @@ struct TokenArgs {
   float *token_score;  // nullable
   int batch, n_q_heads, n_kv_heads, d, block_size, n_blocks_max, max_ctx, n_label, k_b, k_t, dtype;
   int *err;           // the library's device error word
+  const float *scales;  // int8 slab: [B*H_kv][r] channel scales; nullptr for a slab of the K dtype
 };
 // Token score and top-K_t in one launch (one thread-block cluster per group).
 cudaError_t launch_token_select(const TokenArgs &a, cudaStream_t st);

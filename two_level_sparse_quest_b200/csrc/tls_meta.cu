@@ -70,6 +70,52 @@ __global__ void __launch_bounds__(256) build_slab_kernel(MetaArgs a) {
   static_cast<S *>(a.slab)[(static_cast<size_t>(group) * a.max_ctx + t) * a.n_label + c] = v;
 }
 
+// int8 label slab, step 1: per (group, label channel) the largest |K| over the
+// valid tokens, read off the block summary (max(|max|, |min|) of each valid
+// block is the block's largest |K|: exact), then scale = that / 127 (IEEE
+// division).  One CTA per group; thread i takes channel i % r.
+__global__ void __launch_bounds__(256) label_scales_kernel(MetaArgs a, float *scales) {
+  grid_dependency_wait();
+  __shared__ uint32_t amax[64];  // non-negative floats order like their bit patterns
+  const int group = blockIdx.x, r = a.n_label;
+  const int seq = min(max(a.seq_lens[group / a.n_kv_heads], 0), a.max_ctx);
+  const int nb = (seq + a.block_size - 1) / a.block_size;
+  if (threadIdx.x < r) amax[threadIdx.x] = 0u;
+  __syncthreads();
+  const int c = threadIdx.x % r, lanes = blockDim.x / r;
+  const int ch = a.label_idx[c];
+  if (static_cast<int>(threadIdx.x) < lanes * r && ch >= 0 && ch < a.d) {
+    const uint16_t *m = static_cast<const uint16_t *>(a.meta) + static_cast<size_t>(group) * a.n_blocks_max * 2 * a.d;
+    float best = 0.f;
+    for (int blk = threadIdx.x / r; blk < nb; blk += lanes) {
+      const uint16_t *row = m + static_cast<size_t>(blk) * 2 * a.d;
+      best = fmaxf(best, fmaxf(fabsf(bf16_lo(row[ch])), fabsf(bf16_lo(row[a.d + ch]))));
+    }
+    atomicMax(&amax[c], __float_as_uint(best));
+  }
+  __syncthreads();
+  if (threadIdx.x < r) scales[static_cast<size_t>(group) * r + threadIdx.x] = __fdiv_rn(__uint_as_float(amax[threadIdx.x]), 127.0f);
+}
+
+// int8 label slab, step 2: code = round-half-even(K / scale) clamped to
+// [-127, 127] (0 where the scale is 0), decided in fp32; rows t < seq only.
+__global__ void __launch_bounds__(256) build_slab_q8_kernel(MetaArgs a, const float *scales) {
+  grid_dependency_wait();
+  const int group = blockIdx.y;
+  const int seq = min(max(a.seq_lens[group / a.n_kv_heads], 0), a.max_ctx);
+  const long long item = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int t = static_cast<int>(item / a.n_label), c = static_cast<int>(item % a.n_label);
+  if (t >= seq) return;
+  const int ch = a.label_idx[c];
+  const float scale = scales[static_cast<size_t>(group) * a.n_label + c];
+  int code = 0;
+  if (scale > 0.f && ch >= 0 && ch < a.d) {
+    const uint16_t v = static_cast<const uint16_t *>(a.K)[(static_cast<size_t>(group) * a.max_ctx + t) * a.d + ch];
+    code = min(max(__float2int_rn(__fdiv_rn(bf16_lo(v), scale)), -127), 127);
+  }
+  static_cast<int8_t *>(a.slab)[(static_cast<size_t>(group) * a.max_ctx + t) * a.n_label + c] = static_cast<int8_t>(code);
+}
+
 // Append update: CTA (j, group) rebuilds the j-th block touched by the rows
 // [old, new) of the group's sequence from the block's valid rows (max / min
 // over the stored values: exact, so the result equals a rebuild at the new
@@ -162,6 +208,18 @@ cudaError_t launch_build_slab(const MetaArgs &a, cudaStream_t st) {
   dim3 grid(static_cast<unsigned>((items + 255) / 256), a.batch * a.n_kv_heads);
   if (a.dtype == 1) return launch_pdl(build_slab_kernel<BF16>, grid, dim3(256), 0, st, a);
   return launch_pdl(build_slab_kernel<F32>, grid, dim3(256), 0, st, a);
+}
+
+cudaError_t launch_label_scales(const MetaArgs &a, float *scales, cudaStream_t st) {
+  if (a.dtype != 1 || a.n_label > 64 || 256 % a.n_label) return cudaErrorInvalidValue;
+  return launch_pdl(label_scales_kernel, dim3(a.batch * a.n_kv_heads), dim3(256), 0, st, a, scales);
+}
+
+cudaError_t launch_build_slab_q8(const MetaArgs &a, const float *scales, cudaStream_t st) {
+  if (a.dtype != 1) return cudaErrorInvalidValue;
+  const long long items = static_cast<long long>(a.max_ctx) * a.n_label;
+  dim3 grid(static_cast<unsigned>((items + 255) / 256), a.batch * a.n_kv_heads);
+  return launch_pdl(build_slab_q8_kernel, grid, dim3(256), 0, st, a, scales);
 }
 
 }  // namespace tls

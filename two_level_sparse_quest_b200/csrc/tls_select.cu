@@ -197,7 +197,8 @@ __device__ __forceinline__ void score_blocks_max(const BlockScoreArgs &a, int gr
   }
 }
 
-// Qbar_L[c] = sum_h q_h[L[c]] (fp32, heads in order) into qbar[0..r).
+// Qbar_L[c] = sum_h q_h[L[c]] (fp32, heads in order) into qbar[0..r); with an
+// int8 slab the channel's scale is folded in: qbar[c] = scale_c * Qbar_L[c].
 template <typename E>
 __device__ __forceinline__ void fold_label_query(const TokenArgs &a, int group, float *qbar) {
   const int b = group / a.n_kv_heads, g = group % a.n_kv_heads;
@@ -208,20 +209,24 @@ __device__ __forceinline__ void fold_label_query(const TokenArgs &a, int group, 
     if (ch >= 0 && ch < a.d)
       for (int hh = 0; hh < G; ++hh)
         sum += load_elem<E>(a.q, (static_cast<size_t>(b) * a.n_q_heads + g * G + hh) * a.d + ch);
-    qbar[c] = sum;
+    qbar[c] = a.scales ? sum * a.scales[static_cast<size_t>(group) * a.n_label + c] : sum;
   }
 }
 
 // ---------------------------------------------------------------- stage 3 body
 // Scores candidates [c0, c1) of the group (blk[j / bs - jb0] = kept block id,
 // < 0 for none; qbar in shared memory, complete) into keys[j - c0] and hist.
-// RCH: 16-byte chunks per slab row (r * bytes / 16), 1..8.
+// SE: the slab's storage (the K dtype, or I8 codes); RCH: 16-byte chunks per
+// slab row (r * bytes / 16), 1..8.
+template <int RCH, int EPC>
+constexpr int token_min_blocks() { return (RCH > 2 || RCH * EPC > 16) ? 2 : 4; }
+
 template <typename E, int RCH>
 __device__ __forceinline__ void score_tokens(const TokenArgs &a, int group, int seq, int c0, int c1, const int *blk,
                                              int jb0, const float *qbar, uint32_t *keys, int *hist) {
   using S_t = typename E::storage;
   constexpr int EPC = E::kEPC;
-  constexpr int kBatch = RCH <= 4 ? 4 : 2;  // candidates whose rows a thread loads at once
+  constexpr int kBatch = (RCH <= 4 && RCH * EPC <= 32) ? 4 : 2;  // candidates whose rows a thread loads at once
   const int bs = a.block_size, r = a.n_label;
   const int C = a.k_b * bs;
   const bool bs_pow2 = (bs & (bs - 1)) == 0;
@@ -312,8 +317,9 @@ __global__ void __launch_bounds__(kThreads, NCH > 32 ? 2 : 4) block_select_kerne
       [r0](int i) { return r0 + i; }, S, a.err);
 }
 
-template <typename E, int RCH, int CS>
-__global__ void __launch_bounds__(kThreads, RCH > 2 ? 2 : 4) token_select_kernel(TokenArgs a, int per_cta) {
+template <typename E, typename SE, int RCH, int CS>
+__global__ void __launch_bounds__(kThreads, token_min_blocks<RCH, SE::kEPC>())
+    token_select_kernel(TokenArgs a, int per_cta) {
   extern __shared__ uint32_t keys[];  // [per_cta]
   __shared__ int blk[1024];           // block ids of the slice's blocks
   __shared__ float qbar[64];
@@ -331,7 +337,7 @@ __global__ void __launch_bounds__(kThreads, RCH > 2 ? 2 : 4) token_select_kernel
   }
   fold_label_query<E>(a, group, qbar);
   __syncthreads();
-  score_tokens<E, RCH>(a, group, seq, sl.c0, sl.c1, blk, sl.jb0, qbar, keys, S.hist);
+  score_tokens<SE, RCH>(a, group, seq, sl.c0, sl.c1, blk, sl.jb0, qbar, keys, S.hist);
   const int bs = a.block_size, jb0 = sl.jb0, c0 = sl.c0;
   cluster_topk<kThreads, CS, kSliceCap>(
       keys, sl.c1 - sl.c0, a.k_t, a.token_idx + static_cast<size_t>(group) * a.k_t, a.k_t,
@@ -348,8 +354,8 @@ struct StepArgs {
   TokenArgs tok;
 };
 
-template <typename E, int NCH, int RCH, int CS>
-__global__ void __launch_bounds__(kThreads, (NCH > 32 || RCH > 2) ? 2 : 4)
+template <typename E, typename SE, int NCH, int RCH, int CS>
+__global__ void __launch_bounds__(kThreads, NCH > 32 ? 2 : token_min_blocks<RCH, SE::kEPC>())
     select_step_kernel(StepArgs s, int rows_per_cta, int per_cta) {
   extern __shared__ float qpm[];  // [2d] Q^+, Q^-; block keys [rows_per_cta]; token keys [per_cta]
   __shared__ ClusterSelectSmem<CS> SB, ST;
@@ -390,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, (NCH > 32 || RCH > 2) ? 2 : 4)
     blk[i] = (v >= 0 && v < t.n_blocks_max) ? v : -1;
   }
   __syncthreads();
-  score_tokens<E, RCH>(t, group, sq, sl.c0, sl.c1, blk, sl.jb0, qbar, tkeys, ST.hist);
+  score_tokens<SE, RCH>(t, group, sq, sl.c0, sl.c1, blk, sl.jb0, qbar, tkeys, ST.hist);
   const int bs = t.block_size, jb0 = sl.jb0, c0 = sl.c0;
   cluster_topk<kThreads, CS, kSliceCap>(
       tkeys, sl.c1 - sl.c0, t.k_t, t.token_idx + static_cast<size_t>(group) * t.k_t, t.k_t,
@@ -439,26 +445,26 @@ cudaError_t run_block_select(const BlockScoreArgs &a, cudaStream_t st) {
   return run_block_select_agg<E, NCH, false>(a, st);
 }
 
-template <typename E, int RCH>
+template <typename E, typename SE, int RCH>
 cudaError_t run_token_select(const TokenArgs &a, cudaStream_t st) {
   constexpr int CS = kClusterSize;
   const int per = (a.k_b * a.block_size + CS - 1) / CS;  // <= kSliceCap
   const size_t smem = static_cast<size_t>(per) * sizeof(uint32_t);
   static int allowed[64] = {};
-  cudaError_t e = allow_smem(token_select_kernel<E, RCH, CS>, smem, allowed);
+  cudaError_t e = allow_smem(token_select_kernel<E, SE, RCH, CS>, smem, allowed);
   if (e != cudaSuccess) return e;
-  return launch_pdl_cluster(token_select_kernel<E, RCH, CS>, dim3(CS, a.batch * a.n_kv_heads), dim3(kThreads), smem,
+  return launch_pdl_cluster(token_select_kernel<E, SE, RCH, CS>, dim3(CS, a.batch * a.n_kv_heads), dim3(kThreads), smem,
                             st, CS, a, per);
 }
 
-template <typename E, int NCH, int RCH>
+template <typename E, typename SE, int NCH, int RCH>
 cudaError_t run_select_step(const BlockScoreArgs &a, const TokenArgs &t, cudaStream_t st) {
   constexpr int CS = kClusterSize;
   const int rows = (a.n_blocks_max + CS - 1) / CS;
   const int per = (t.k_b * t.block_size + CS - 1) / CS;
   const size_t smem = 2 * static_cast<size_t>(a.d) * sizeof(float) +
                       (static_cast<size_t>(rows) + static_cast<size_t>(per)) * sizeof(uint32_t);
-  auto kern = select_step_kernel<E, NCH, RCH, CS>;
+  auto kern = select_step_kernel<E, SE, NCH, RCH, CS>;
   static int allowed[64] = {};
   cudaError_t e = allow_smem(kern, smem, allowed);
   if (e != cudaSuccess) return e;
@@ -468,11 +474,22 @@ cudaError_t run_select_step(const BlockScoreArgs &a, const TokenArgs &t, cudaStr
 
 template <typename E, int NCH>
 cudaError_t step_by_rch(const BlockScoreArgs &a, const TokenArgs &t, cudaStream_t st) {
+  if constexpr (sizeof(typename E::storage) == 2) {
+    if (t.scales) {  // int8 label slab
+      switch (t.n_label / 16) {
+        case 1: return run_select_step<E, I8, NCH, 1>(a, t, st);
+        case 2: return run_select_step<E, I8, NCH, 2>(a, t, st);
+        case 4: return run_select_step<E, I8, NCH, 4>(a, t, st);
+      }
+      return cudaErrorInvalidValue;
+    }
+  }
+  if (t.scales) return cudaErrorInvalidValue;
   switch (t.n_label * E::kBytes / 16) {
-    case 1: return run_select_step<E, NCH, 1>(a, t, st);
-    case 2: return run_select_step<E, NCH, 2>(a, t, st);
-    case 4: return run_select_step<E, NCH, 4>(a, t, st);
-    case 8: return run_select_step<E, NCH, 8>(a, t, st);
+    case 1: return run_select_step<E, E, NCH, 1>(a, t, st);
+    case 2: return run_select_step<E, E, NCH, 2>(a, t, st);
+    case 4: return run_select_step<E, E, NCH, 4>(a, t, st);
+    case 8: return run_select_step<E, E, NCH, 8>(a, t, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -497,12 +514,21 @@ cudaError_t launch_block_select(const BlockScoreArgs &a, cudaStream_t st) {
 }
 
 cudaError_t launch_token_select(const TokenArgs &a, cudaStream_t st) {
+  if (a.scales) {  // int8 label slab (bf16 queries)
+    if (a.dtype != 1) return cudaErrorInvalidValue;
+    switch (a.n_label / 16) {
+      case 1: return run_token_select<BF16, I8, 1>(a, st);
+      case 2: return run_token_select<BF16, I8, 2>(a, st);
+      case 4: return run_token_select<BF16, I8, 4>(a, st);
+    }
+    return cudaErrorInvalidValue;
+  }
   const int rch = a.n_label * (a.dtype == 1 ? 2 : 4) / 16;
   switch (rch) {
-    case 1: return a.dtype == 1 ? run_token_select<BF16, 1>(a, st) : run_token_select<F32, 1>(a, st);
-    case 2: return a.dtype == 1 ? run_token_select<BF16, 2>(a, st) : run_token_select<F32, 2>(a, st);
-    case 4: return a.dtype == 1 ? run_token_select<BF16, 4>(a, st) : run_token_select<F32, 4>(a, st);
-    case 8: return a.dtype == 1 ? run_token_select<BF16, 8>(a, st) : run_token_select<F32, 8>(a, st);
+    case 1: return a.dtype == 1 ? run_token_select<BF16, BF16, 1>(a, st) : run_token_select<F32, F32, 1>(a, st);
+    case 2: return a.dtype == 1 ? run_token_select<BF16, BF16, 2>(a, st) : run_token_select<F32, F32, 2>(a, st);
+    case 4: return a.dtype == 1 ? run_token_select<BF16, BF16, 4>(a, st) : run_token_select<F32, F32, 4>(a, st);
+    case 8: return a.dtype == 1 ? run_token_select<BF16, BF16, 8>(a, st) : run_token_select<F32, F32, 8>(a, st);
   }
   return cudaErrorInvalidValue;
 }

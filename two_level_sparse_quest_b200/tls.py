@@ -31,14 +31,15 @@ STATUS_NAMES = {0: "TLS_OK", 1: "TLS_ERR_INVALID_ARG", 2: "TLS_ERR_UNSUPPORTED",
 EXPORTED = ("tls_version", "tls_last_error", "tls_workspace_size", "tls_build_block_meta", "tls_block_score_topk",
             "tls_token_score_topk", "tls_sparse_attn_decode", "tls_sparse_attn_decode_paged", "tls_offload_reset",
             "tls_prefetch_diff", "tls_wait_event", "tls_block_score_topk_noalloc", "tls_device_error", "tls_select_step",
-            "tls_append_tokens")
+            "tls_append_tokens", "tls_slab_bytes")
 
 
 class TlsShape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "batch", "n_q_heads", "n_kv_heads", "d_qk", "d_v", "v_is_k_prefix", "block_size", "n_label",
         "k_b", "k_t", "max_ctx", "kv_dtype", "out_dtype")] + [("softmax_scale", ctypes.c_float),
-                                                               ("block_agg", ctypes.c_int32)]
+                                                               ("block_agg", ctypes.c_int32),
+                                                               ("slab_bits", ctypes.c_int32)]
 
     def __repr__(self):
         return "TlsShape(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
@@ -70,6 +71,7 @@ _sigs = {
     "tls_device_error": ([ctypes.POINTER(_i32), _i32], ctypes.c_int),
     "tls_select_step": ([_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "tls_append_tokens": ([_S, _P, _P, _P, _i32, _P, _P, _P, _P], ctypes.c_int),
+    "tls_slab_bytes": ([_S], _sz),
 }
 for _name, (_args, _ret) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -79,7 +81,7 @@ for _name, (_args, _ret) in _sigs.items():
 
 def make_shape(batch, n_q_heads, n_kv_heads, d_qk, d_v, block_size, n_label, k_b, k_t, max_ctx, kv_dtype,
                out_dtype=TLS_F32, v_is_k_prefix=False, softmax_scale: Optional[float] = None,
-               block_agg: int = 0) -> TlsShape:
+               block_agg: int = 0, slab_bits: int = 0) -> TlsShape:
     s = TlsShape()
     s.batch, s.n_q_heads, s.n_kv_heads = batch, n_q_heads, n_kv_heads
     s.d_qk, s.d_v, s.v_is_k_prefix = d_qk, d_v, int(bool(v_is_k_prefix))
@@ -87,13 +89,15 @@ def make_shape(batch, n_q_heads, n_kv_heads, d_qk, d_v, block_size, n_label, k_b
     s.kv_dtype, s.out_dtype = kv_dtype, out_dtype
     s.softmax_scale = (1.0 / math.sqrt(d_qk)) if softmax_scale is None else softmax_scale
     s.block_agg = int(block_agg)
+    s.slab_bits = int(slab_bits)
     return s
 
 
 def shape_from_workload(w, out_dtype=TLS_F32, **over) -> TlsShape:
     kw = dict(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, d_qk=w.d_qk, d_v=w.d_v,
               block_size=w.block_size, n_label=w.n_label, k_b=w.k_b, k_t=w.k_t, max_ctx=w.ctx, kv_dtype=w.dtype,
-              out_dtype=out_dtype, v_is_k_prefix=w.v_is_k_prefix, block_agg=getattr(w, "block_agg", 0))
+              out_dtype=out_dtype, v_is_k_prefix=w.v_is_k_prefix, block_agg=getattr(w, "block_agg", 0),
+              slab_bits=getattr(w, "slab_bits", 0))
     kw.update(over)
     return make_shape(**kw)
 
@@ -143,6 +147,13 @@ def tls_workspace_size(shape: TlsShape) -> int:
     n = _lib.tls_workspace_size(ctypes.byref(shape))
     if n == 0:
         raise TlsError(TLS_ERR_UNSUPPORTED, f"tls_workspace_size: {tls_last_error()}")
+    return n
+
+
+def tls_slab_bytes(shape: TlsShape) -> int:
+    n = _lib.tls_slab_bytes(ctypes.byref(shape))
+    if n == 0:
+        raise TlsError(TLS_ERR_UNSUPPORTED, f"tls_slab_bytes: {tls_last_error()}")
     return n
 
 
