@@ -125,6 +125,17 @@ def test_block_aggregation_field_is_checked(T):
     assert call_block(T, mla) == T.TLS_ERR_UNSUPPORTED
 
 
+def test_group_sizes(T):
+    for G in (1, 2, 4, 8, 16, 32, 64):  # host-side plan only: nothing is launched
+        assert T.tls_workspace_size(good_shape(T, n_q_heads=G, n_kv_heads=1)) > 0
+        assert T.tls_workspace_size(good_shape(T, n_q_heads=G, n_kv_heads=1, d_qk=64, d_v=64)) > 0
+    st = call_block(T, good_shape(T, n_q_heads=24, n_kv_heads=1))
+    assert st == T.TLS_ERR_UNSUPPORTED and "group size" in T.tls_last_error()
+    mq = good_shape(T, n_q_heads=16, n_kv_heads=1)
+    mq.block_agg = 1
+    assert call_block(T, mq) == T.TLS_ERR_UNSUPPORTED and "up to 8 heads" in T.tls_last_error()
+
+
 def test_int8_slab_field_and_size(T):
     s = good_shape(T)
     n0 = T.tls_slab_bytes(s)

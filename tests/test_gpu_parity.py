@@ -46,6 +46,17 @@ SMALL = {
     "block_size_16_odd_ctx": (W.WORKLOADS["gqa48k_bf16"].with_(block_size=16, ctx=1999, k_b=40, k_t=333), None),
     "mla_small": (W.WORKLOADS["mla64k_b4_bf16"].with_(batch=2, ctx=4096, k_b=16, k_t=300, n_needles=4),
                   [4096, 3000]),
+    # shape sweep: MHA (one query head per KV head) and MQA (one KV head for
+    # 16, 32 or 64 query heads: units of 16 heads on the warp-MMA kernel)
+    "mha_h16": (W.WORKLOADS["gqa48k_bf16"].with_(n_q_heads=16, n_kv_heads=16, ctx=2048, k_b=16, k_t=200), None),
+    "mqa_g16": (W.WORKLOADS["gqa48k_bf16"].with_(batch=2, n_q_heads=16, n_kv_heads=1, ctx=4096, k_b=24, k_t=300),
+                [4096, 2999]),
+    "mqa_g32": (W.WORKLOADS["gqa48k_bf16"].with_(batch=2, n_q_heads=32, n_kv_heads=1, ctx=4096, k_b=24, k_t=300),
+                [4096, 1777]),
+    "mqa_g64_d64": (W.WORKLOADS["gqa48k_bf16"].with_(batch=3, n_q_heads=64, n_kv_heads=1, d_qk=64, d_v=64, ctx=3000,
+                                                     k_b=20, k_t=211), [3000, 17, 2500]),
+    "mqa_g32_f32": (W.WORKLOADS["tiny_gqa4k_f32"].with_(batch=2, n_q_heads=32, n_kv_heads=1, ctx=1000, k_b=8,
+                                                        k_t=100), [1000, 640]),
 }
 
 
@@ -147,7 +158,8 @@ def test_alternative_attention_kernels_parity(impl):
     import sys
 
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    cases = ["gqa_bf16_small", "gqa_bf16_g8", "mla_small"] if impl == "cuda_core" else ["gqa_bf16_small", "gqa_bf16_g8"]
+    cases = (["gqa_bf16_small", "gqa_bf16_g8", "mla_small", "mqa_g32", "mqa_g64_d64"] if impl == "cuda_core"
+             else ["gqa_bf16_small", "gqa_bf16_g8"])
     code = (
         "import sys; sys.path.insert(0, %r)\n"
         "from tests import test_gpu_parity as t, _parity as P\n"

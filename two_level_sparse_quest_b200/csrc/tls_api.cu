@@ -79,7 +79,10 @@ tls_status check_shape(const tls_shape *s) {
   } else {
     if (s->d_qk != s->d_v || (s->d_qk != 64 && s->d_qk != 128))
       return fail(TLS_ERR_UNSUPPORTED, "GQA supports d_qk = d_v in {64, 128} (got %d, %d)", s->d_qk, s->d_v);
-    if (G != 1 && G != 2 && G != 4 && G != 8) return fail(TLS_ERR_UNSUPPORTED, "GQA group size %d not in {1,2,4,8}", G);
+    if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16 && G != 32 && G != 64)
+      return fail(TLS_ERR_UNSUPPORTED, "GQA group size %d not in {1,2,4,8,16,32,64}", G);
+    if (s->block_agg == 1 && G > 8)
+      return fail(TLS_ERR_UNSUPPORTED, "max-over-heads block aggregation supports groups of up to 8 heads");
   }
   if (n_blocks_max(s) > tls::kMaxSelectKeys)
     return fail(TLS_ERR_UNSUPPORTED, "ceil(max_ctx / block_size) = %d > %d", n_blocks_max(s), tls::kMaxSelectKeys);

@@ -393,11 +393,12 @@ bool pick_variant(const AttnArgs &a, Variant *v) {
     return true;
   }
   if (a.d_qk != a.d_v || (a.d_qk != 64 && a.d_qk != 128)) return false;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return false;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16 && G != 32 && G != 64) return false;
+  const int hc = G < 8 ? G : 8;  // larger groups run as units of 8 heads
   int w;
-  if (a.dtype == 1) w = a.d_qk == 128 ? gqa_warps<BF16, 128>(G) : gqa_warps<BF16, 64>(G);
-  else w = a.d_qk == 128 ? gqa_warps<F32, 128>(G) : gqa_warps<F32, 64>(G);
-  *v = {w, G};
+  if (a.dtype == 1) w = a.d_qk == 128 ? gqa_warps<BF16, 128>(hc) : gqa_warps<BF16, 64>(hc);
+  else w = a.d_qk == 128 ? gqa_warps<F32, 128>(hc) : gqa_warps<F32, 64>(hc);
+  *v = {w, hc};
   return true;
 }
 
@@ -464,7 +465,10 @@ bool attn_plan(const AttnArgs &a, AttnPlan *p) {
   p->impl = mma ? 2 : 0;
   Variant v;
   if (!pick_variant(a, &v)) return false;
-  if (mma) v.warps = attn_mma_warps(a);
+  if (mma) {
+    v.warps = attn_mma_warps(a);
+    v.head_chunk = attn_mma_head_chunk(a);
+  }
   const int G = a.n_q_heads / a.n_kv_heads;
   p->warps_per_cta = v.warps;
   p->tokens_per_tile = kTT;
@@ -515,6 +519,7 @@ cudaError_t launch_attention_merge(const AttnArgs &a, const AttnPlan &p, cudaStr
     case 2: return dv == 128 ? run_merge<128, 2>(a, p, st) : run_merge<64, 2>(a, p, st);
     case 4: return dv == 128 ? run_merge<128, 4>(a, p, st) : run_merge<64, 4>(a, p, st);
     case 8: return dv == 128 ? run_merge<128, 8>(a, p, st) : run_merge<64, 8>(a, p, st);
+    case 16: return dv == 128 ? run_merge<128, 16>(a, p, st) : run_merge<64, 16>(a, p, st);
   }
   return cudaErrorInvalidValue;
 }

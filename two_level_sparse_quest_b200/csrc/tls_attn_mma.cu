@@ -9,9 +9,11 @@
 // tiles per warp, a private cp.async ring per warp, partial (max, sum, o)
 // per unit and piece, log-sum-exp merge kernel).  Per tile, one warp:
 //   S = Q K^T   mma m16n8k16 (bf16 in, fp32 accumulate): M = the unit's heads
-//               (rows padded to 16; Q fragments stay in registers for the
-//               unit), N = 8 tokens x 2, K = d in steps of 16; K fragments come
-//               from the XOR-swizzled stage buffer through ldmatrix.
+//               (up to 8 heads use rows 0-7 and leave rows 8-15 zero; a unit
+//               of 16 heads fills all 16 rows, two per lane quad; Q fragments
+//               stay in registers for the unit), N = 8 tokens x 2, K = d in
+//               steps of 16; K fragments come from the XOR-swizzled stage
+//               buffer through ldmatrix.
 //   online softmax in the log2 domain on the S accumulators (a row = a head
 //               lives in one lane quad: max and sum are two quad shuffles).
 //   O += P V    the S accumulator layout of two 8-token blocks is exactly the
@@ -21,7 +23,9 @@
 //               swizzled stage buffer through ldmatrix.trans.
 // The tensor cores replace ~40 FMA-pipe instructions per token and head
 // group with 3 MMAs, which moves the kernel from issue-bound to HBM-bound on
-// the gathered rows.
+// the gathered rows.  Groups of 32 or 64 heads (MQA-like shapes) are cut
+// into units of 16 heads that gather the group's rows each; the units of one
+// group sit in adjacent warps, so the repeated gathers mostly hit L2.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -80,6 +84,23 @@ __device__ __forceinline__ void mma_rows(float (&c)[2], uint32_t a0, uint32_t a2
       : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1), "f"(0.f), "f"(0.f));
 }
 
+// c[0..3] += A B over all 16 rows (rows lane/4 and lane/4 + 8).
+__device__ __forceinline__ void mma_full(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// R = 1: rows lane/4 only (A fragment {a0, a2}); R = 2: both row halves
+// (A fragment {a0, a1, a2, a3}); c holds 2 R accumulators.
+template <int R>
+__device__ __forceinline__ void mma_r(float (&c)[2 * R], const uint32_t (&a)[2 * R], uint32_t b0, uint32_t b1) {
+  if constexpr (R == 1) mma_rows(c, a[0], a[1], b0, b1);
+  else mma_full(c, a[0], a[1], a[2], a[3], b0, b1);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t *>(&v);
@@ -95,7 +116,8 @@ __global__ void __launch_bounds__(MmaLayout<D, NS>::W * 32, 1) attn_mma_kernel(A
   using L = MmaLayout<D, NS>;
   constexpr int KS = D / 16;  // k-steps of S = Q K^T
   constexpr int NB = D / 8;   // 8-channel blocks of O
-  static_assert(HG <= 8, "a head group fits the first 8 MMA rows");
+  constexpr int R = HG > 8 ? 2 : 1;  // MMA rows per lane: lane/4 (and lane/4 + 8)
+  static_assert(HG <= 16, "a unit's heads fit the 16 MMA rows");
   extern __shared__ __align__(128) unsigned char smem[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned char *wbase = smem + warp * L::kWarpBytes;
@@ -114,15 +136,21 @@ __global__ void __launch_bounds__(MmaLayout<D, NS>::W * 32, 1) attn_mma_kernel(A
   const int Gt = a.n_q_heads / a.n_kv_heads;
 
   // Gather the K and V rows of tile t into stage st (the caller commits).
-  // Issue cursor: tile iss_t (its unit = group, tile within the group, ring
-  // stage) advances by counting, so no integer division sits on the per-tile
-  // path.  A unit is one GQA group (the plan has one head chunk per group).
-  int iss_t = t_begin, iss_group = t_begin / p.tiles_per_group, iss_tile = t_begin % p.tiles_per_group, iss_st = 0;
+  // Issue cursor: tile iss_t (its group, head chunk, tile within the unit,
+  // ring stage) advances by counting, so no integer division sits on the
+  // per-tile path.  A unit is one head chunk of one group.
+  const int nhc = p.n_head_chunks;
+  const int unit0 = t_begin / p.tiles_per_group;
+  int iss_t = t_begin, iss_group = unit0 / nhc, iss_hc = unit0 % nhc, iss_tile = t_begin % p.tiles_per_group,
+      iss_st = 0;
   auto issue_next = [&]() {
     const int t = iss_t, st = iss_st, tile = iss_tile, group = iss_group;
     if (++iss_tile == p.tiles_per_group) {
       iss_tile = 0;
-      ++iss_group;
+      if (++iss_hc == nhc) {
+        iss_hc = 0;
+        ++iss_group;
+      }
     }
     ++iss_t;
     if (++iss_st == NS) iss_st = 0;
@@ -164,46 +192,58 @@ __global__ void __launch_bounds__(MmaLayout<D, NS>::W * 32, 1) attn_mma_kernel(A
     }
   };
 
-  const int g = lane >> 2;          // MMA row of this lane = head within the unit
+  const int g = lane >> 2;          // MMA row of this lane = head within the unit (and g + 8 when R = 2)
   const int tq = 2 * (lane & 3);    // first of this lane's token (or channel) pair
-  uint32_t qa[KS][2];               // A fragments of Q (rows g; rows g + 8 are zero)
-  float o[NB][2];                   // O[g][8j + tq .. + 1]
-  float m_run = -INFINITY, l_run = 0.f;
+  // A fragments of Q: R = 1 {rows g: ch tq, ch 8 + tq}; R = 2 {g, g + 8, g: 8 + tq, g + 8: 8 + tq}
+  uint32_t qa[KS][2 * R];
+  float o[NB][2 * R];               // O[g (+ 8 r)][8j + tq .. + 1] at [j][2r .. 2r + 1]
+  float m_run[R], l_run[R];
   int cur_unit = -1;
 
   auto flush = [&](int unit) {
-    float lt = l_run;
-    lt += __shfl_xor_sync(0xffffffffu, lt, 1);
-    lt += __shfl_xor_sync(0xffffffffu, lt, 2);
     const int first = (unit * p.tiles_per_group) / p.tiles_per_warp;
     const int piece = gw - first;
     const size_t units = static_cast<size_t>(a.batch) * a.n_kv_heads * p.n_head_chunks;
     float *ml = a.part + (static_cast<size_t>(unit) * p.max_pieces + piece) * HG * 2;
     float *po = a.part + units * p.max_pieces * HG * 2 + (static_cast<size_t>(unit) * p.max_pieces + piece) * HG * D;
-    if (g < HG) {
-      if ((lane & 3) == 0) {
-        ml[g * 2] = m_run;
-        ml[g * 2 + 1] = lt;
-      }
 #pragma unroll
-      for (int j = 0; j < NB; ++j)
-        *reinterpret_cast<float2 *>(po + g * D + 8 * j + tq) = make_float2(o[j][0], o[j][1]);
+    for (int r = 0; r < R; ++r) {
+      float lt = l_run[r];
+      lt += __shfl_xor_sync(0xffffffffu, lt, 1);
+      lt += __shfl_xor_sync(0xffffffffu, lt, 2);
+      const int h = g + 8 * r;
+      if (h < HG) {
+        if ((lane & 3) == 0) {
+          ml[h * 2] = m_run[r];
+          ml[h * 2 + 1] = lt;
+        }
+#pragma unroll
+        for (int j = 0; j < NB; ++j)
+          *reinterpret_cast<float2 *>(po + h * D + 8 * j + tq) = make_float2(o[j][2 * r], o[j][2 * r + 1]);
+      }
     }
   };
 
-  auto start_unit = [&](int unit) {  // unit = group
-    const int b = unit / a.n_kv_heads, gk = unit % a.n_kv_heads;
+  auto start_unit = [&](int unit) {  // unit = group * n_head_chunks + head chunk
+    const int group = unit / nhc, hc = unit % nhc;
+    const int b = group / a.n_kv_heads, gk = group % a.n_kv_heads;
     const uint32_t *q = static_cast<const uint32_t *>(a.q);
-    const size_t row = (static_cast<size_t>(b) * a.n_q_heads + gk * Gt + g) * D;
 #pragma unroll
-    for (int kk = 0; kk < KS; ++kk) {
-      qa[kk][0] = g < HG ? q[(row + 16 * kk + tq) / 2] : 0u;
-      qa[kk][1] = g < HG ? q[(row + 16 * kk + 8 + tq) / 2] : 0u;
+    for (int r = 0; r < R; ++r) {
+      const int h = g + 8 * r;
+      const size_t row = (static_cast<size_t>(b) * a.n_q_heads + gk * Gt + hc * HG + h) * D;
+#pragma unroll
+      for (int kk = 0; kk < KS; ++kk) {
+        qa[kk][r] = h < HG ? q[(row + 16 * kk + tq) / 2] : 0u;
+        qa[kk][R + r] = h < HG ? q[(row + 16 * kk + 8 + tq) / 2] : 0u;
+      }
+      m_run[r] = -INFINITY;
+      l_run[r] = 0.f;
     }
 #pragma unroll
-    for (int j = 0; j < NB; ++j) o[j][0] = o[j][1] = 0.f;
-    m_run = -INFINITY;
-    l_run = 0.f;
+    for (int j = 0; j < NB; ++j)
+#pragma unroll
+      for (int i = 0; i < 2 * R; ++i) o[j][i] = 0.f;
   };
 
   const int mi = lane >> 3, mr = lane & 7;  // ldmatrix: matrix index and row of this lane's address
@@ -229,8 +269,10 @@ __global__ void __launch_bounds__(MmaLayout<D, NS>::W * 32, 1) attn_mma_kernel(A
     const unsigned char *Vs = Ks + kMT * L::RB;
     const uint32_t vmask = Mask[st];
 
-    // ---- S = Q K^T: tokens 0-7 -> s0, 8-15 -> s1
-    float s0[2] = {0.f, 0.f}, s1[2] = {0.f, 0.f};
+    // ---- S = Q K^T: tokens 0-7 -> s0, 8-15 -> s1 (row g at [0..1], row g + 8 at [2..3])
+    float s0[2 * R], s1[2 * R];
+#pragma unroll
+    for (int i = 0; i < 2 * R; ++i) s0[i] = s1[i] = 0.f;
     {
       const int tok = (mi >> 1) * 8 + mr;
       const uint32_t rowa = smem_addr(Ks + tok * L::RB);
@@ -239,37 +281,52 @@ __global__ void __launch_bounds__(MmaLayout<D, NS>::W * 32, 1) attn_mma_kernel(A
         const int ch = 2 * kk + (mi & 1);
         uint32_t b0, b1, b2, b3;
         ldsm_x4(rowa + ((ch ^ (tok & 7)) << 4), b0, b1, b2, b3);
-        mma_rows(s0, qa[kk][0], qa[kk][1], b0, b1);
-        mma_rows(s1, qa[kk][0], qa[kk][1], b2, b3);
+        mma_r<R>(s0, qa[kk], b0, b1);
+        mma_r<R>(s1, qa[kk], b2, b3);
       }
     }
     // ---- online softmax, log2 domain; lanes of a quad share a row (head)
-    float sc[4] = {s0[0], s0[1], s1[0], s1[1]};
     const int tk[4] = {tq, tq + 1, 8 + tq, 9 + tq};
+    float alpha[R], pr[R][4];
+    bool rescale = false;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) sc[i] = ((vmask >> tk[i]) & 1u) ? sc[i] * a.scale_log2 : -INFINITY;
-    float mt = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
-    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
-    mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
-    const float mn = fmaxf(m_run, mt);
-    float alpha = 1.f, pr[4] = {0.f, 0.f, 0.f, 0.f};
-    if (mn != -INFINITY) {
-      alpha = ex2(m_run - mn);
+    for (int r = 0; r < R; ++r) {
+      float sc[4] = {s0[2 * r], s0[2 * r + 1], s1[2 * r], s1[2 * r + 1]};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) pr[i] = ex2(sc[i] - mn);
-    }
-    l_run = l_run * alpha + ((pr[0] + pr[1]) + (pr[2] + pr[3]));
-    m_run = mn;
-    if (__any_sync(0xffffffffu, alpha != 1.f)) {
+      for (int i = 0; i < 4; ++i) sc[i] = ((vmask >> tk[i]) & 1u) ? sc[i] * a.scale_log2 : -INFINITY;
+      float mt = fmaxf(fmaxf(sc[0], sc[1]), fmaxf(sc[2], sc[3]));
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 1));
+      mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 2));
+      const float mn = fmaxf(m_run[r], mt);
+      alpha[r] = 1.f;
 #pragma unroll
-      for (int j = 0; j < NB; ++j) {
-        o[j][0] *= alpha;
-        o[j][1] *= alpha;
+      for (int i = 0; i < 4; ++i) pr[r][i] = 0.f;
+      if (mn != -INFINITY) {
+        alpha[r] = ex2(m_run[r] - mn);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) pr[r][i] = ex2(sc[i] - mn);
       }
+      l_run[r] = l_run[r] * alpha[r] + ((pr[r][0] + pr[r][1]) + (pr[r][2] + pr[r][3]));
+      m_run[r] = mn;
+      rescale |= alpha[r] != 1.f;
     }
-    uint32_t ph0, pl0, ph1, pl1;  // P over tokens tq..tq+1 (0) and 8+tq..9+tq (1), hi and lo parts
-    split_bf16(pr[0], pr[1], ph0, pl0);
-    split_bf16(pr[2], pr[3], ph1, pl1);
+    if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+      for (int j = 0; j < NB; ++j)
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          o[j][2 * r] *= alpha[r];
+          o[j][2 * r + 1] *= alpha[r];
+        }
+    }
+    // P as the A operand over 16 tokens, hi and lo parts: the same fragment
+    // order as Q ({row g: tokens tq.., (row g + 8: tokens tq..), row g: 8 + tq.., (row g + 8: 8 + tq..)})
+    uint32_t ph[2 * R], pl[2 * R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      split_bf16(pr[r][0], pr[r][1], ph[r], pl[r]);
+      split_bf16(pr[r][2], pr[r][3], ph[R + r], pl[R + r]);
+    }
     // ---- O += P V
     {
       const int tok = (mi & 1) * 8 + mr;
@@ -279,10 +336,10 @@ __global__ void __launch_bounds__(MmaLayout<D, NS>::W * 32, 1) attn_mma_kernel(A
         const int ch = j + (mi >> 1);
         uint32_t v0, v1, v2, v3;
         ldsm_x4_t(rowa + ((ch ^ (tok & 7)) << 4), v0, v1, v2, v3);
-        mma_rows(o[j], ph0, ph1, v0, v1);
-        mma_rows(o[j], pl0, pl1, v0, v1);
-        mma_rows(o[j + 1], ph0, ph1, v2, v3);
-        mma_rows(o[j + 1], pl0, pl1, v2, v3);
+        mma_r<R>(o[j], ph, v0, v1);
+        mma_r<R>(o[j], pl, v0, v1);
+        mma_r<R>(o[j + 1], ph, v2, v3);
+        mma_r<R>(o[j + 1], pl, v2, v3);
       }
     }
     __syncwarp();
@@ -318,6 +375,7 @@ cudaError_t dispatch_mma(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) 
     case 2: return run_mma<D, 2, PAGED>(a, p, st);
     case 4: return run_mma<D, 4, PAGED>(a, p, st);
     case 8: return run_mma<D, 8, PAGED>(a, p, st);
+    case 16: return run_mma<D, 16, PAGED>(a, p, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -327,15 +385,16 @@ cudaError_t dispatch_mma(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) 
 bool attn_mma_supported(const AttnArgs &a) {
   const int G = a.n_q_heads / a.n_kv_heads;
   return a.dtype == 1 && !a.v_is_k_prefix && a.d_qk == a.d_v && (a.d_qk == 64 || a.d_qk == 128) &&
-         (G == 1 || G == 2 || G == 4 || G == 8);
+         (G == 1 || G == 2 || G == 4 || G == 8 || G == 16 || G == 32 || G == 64);
 }
+
+int attn_mma_head_chunk(const AttnArgs &a) { return std::min(a.n_q_heads / a.n_kv_heads, 16); }
 
 int attn_mma_warps(const AttnArgs &a) {
   return a.d_qk == 64 ? MmaLayout<64, kMmaStages>::W : MmaLayout<128, kMmaStages>::W;
 }
 
 cudaError_t launch_attention_mma(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) {
-  if (p.n_head_chunks != 1) return cudaErrorInvalidValue;  // the kernel takes a unit to be a whole group
   if (a.d_qk == 128) return a.paged ? dispatch_mma<128, true>(a, p, st) : dispatch_mma<128, false>(a, p, st);
   return a.paged ? dispatch_mma<64, true>(a, p, st) : dispatch_mma<64, false>(a, p, st);
 }

@@ -138,6 +138,8 @@ bool attn_mla_supported(const AttnArgs &a);
 cudaError_t launch_attention_mla(const AttnArgs &a, const AttnPlan &p, cudaStream_t st);
 bool attn_mma_supported(const AttnArgs &a);
 int attn_mma_warps(const AttnArgs &a);
+// Heads per unit of the warp-MMA kernel: the group, or 16 for larger groups.
+int attn_mma_head_chunk(const AttnArgs &a);
 cudaError_t launch_attention_mma(const AttnArgs &a, const AttnPlan &p, cudaStream_t st);
 bool attn_tc_supported(const AttnArgs &a);
 bool attn_tc_plan(const AttnArgs &a, AttnPlan *p);
