@@ -129,9 +129,10 @@ TLS_API size_t tls_slab_bytes(const tls_shape *s);
  *   slab_out   device [B][H_kv][max_ctx][n_label]: slab[.., t, c] = K[.., t, label_idx[c]]
  *              for t < seq_len (other rows untouched); may be NULL to skip.
  *              slab_bits 8 (the quantised variant): tls_slab_bytes(s) bytes holding
- *              the codes round-half-even(K / scale) clamped to [-127, 127] (rows
- *              >= seq_len: 0) and the scales max|K[.., t < seq_len, L_c]| / 127,
- *              both decided in fp32 (the max comes from the block summary). */
+ *              the codes round-half-even(K / scale) clamped to [-127, 127] (0 where
+ *              the scale is 0; rows >= seq_len untouched) and the scales
+ *              max|K[.., t < seq_len, L_c]| / 127, both decided in fp32 (the max
+ *              comes from the block summary, so meta_out is written first). */
 TLS_API tls_status tls_build_block_meta(const tls_shape *s, const void *K, const int32_t *seq_lens,
                                 const int32_t *label_idx, void *meta_out, void *slab_out, void *stream);
 
@@ -179,7 +180,9 @@ TLS_API tls_status tls_block_score_topk(const tls_shape *s, const void *q, const
  * for the candidates t = block_idx[j / bs] * bs + j % bs (j < k_b * bs) with
  * block id >= 0 and t < seq_len.  fp32 accumulation; ranked on fp32, equal
  * scores to the lower token index.
- *   slab            device [B][H_kv][max_ctx][n_label] (tls_build_block_meta)
+ *   slab            device [B][H_kv][max_ctx][n_label] (tls_build_block_meta); with
+ *                   slab_bits 8 the int8 slab, and slab[t][c] reads scale_c * code
+ *                   (the kernel multiplies scale_c into the summed query channel)
  *   label_idx       device int32 [n_label]
  *   block_idx       device int32 [B][H_kv][k_b] (ids < 0 are skipped)
  *   token_idx_out   device int32 [B][H_kv][k_t], ascending token positions, -1 padded
