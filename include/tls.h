@@ -90,12 +90,14 @@ typedef struct tls_shape {
 
 /* Supported shapes (others return TLS_ERR_UNSUPPORTED):
  *   GQA/MQA/MHA: v_is_k_prefix = 0, kv_dtype F32 or BF16, d_qk = d_v in {64, 128},
- *                G = n_q_heads / n_kv_heads in {1, 2, 4, 8};
+ *                G = n_q_heads / n_kv_heads in {1, 2, 4, 8, 16, 32, 64} (block_agg 1:
+ *                G <= 8);
  *   MLA:         v_is_k_prefix = 1, kv_dtype BF16, d_qk = 576, d_v = 512,
  *                G a multiple of 4 up to 128;
  *   block_size >= 1, ceil(max_ctx / bs) <= 16384 blocks, 1 <= k_b <= 1024,
  *   k_b * bs <= 16384 candidates, k_t >= 1, B * H_kv <= 65535;
- *   n_label in {8, 16, 32, 64} (BF16) or {4, 8, 16, 32} (F32). */
+ *   n_label in {8, 16, 32, 64} (BF16) or {4, 8, 16, 32} (F32);
+ *   slab_bits 0, or 8 with BF16 keys and n_label in {16, 32, 64}. */
 
 /* Library version string, e.g. "tls 0.1 sm_100a". */
 TLS_API const char *tls_version(void);
