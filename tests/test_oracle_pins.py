@@ -314,6 +314,27 @@ def test_attention_is_invariant_to_selection_order_and_padding():
     np.testing.assert_allclose(la, lb, rtol=1e-14)
 
 
+def test_attention_shift_invariance_with_large_logits():
+    # Adding one vector v to every key moves every logit of head h by
+    # tau * q_h.v: the output stays the same and lse moves by exactly that
+    # amount, even when the shifted logits (~2048) would overflow exp in fp64
+    # without the running-max subtraction.  Grid values keep every sum exact.
+    sh = Sh(n_q_heads=2, n_kv_heads=1, ctx=16, d_qk=4, d_v=4, k_t=6)
+    rng = np.random.default_rng(5)
+    q = (rng.integers(-8, 9, (1, 2, 4)) / 8).astype(np.float32)
+    q[0, :, 0] = [1.0, 0.5]
+    K = (rng.integers(-16, 17, (1, 1, 16, 4)) / 16).astype(np.float32)
+    V = rng.standard_normal((1, 1, 16, 4)).astype(np.float32)
+    shift = np.array([2048.0, 0.0, 0.0, 0.0], np.float32)
+    s = O.shape_of(sh, softmax_scale=1.0)
+    idx = np.array([[[0, 3, 5, 8, 11, 15]]], np.int32)
+    a, la = O.attention(s, q, K, V, idx)
+    b, lb = O.attention(s, q, np.ascontiguousarray(K + shift), V, idx)
+    assert np.isfinite(b).all() and np.isfinite(lb).all()
+    np.testing.assert_allclose(b, a, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose((lb - la)[0], q[0, :, 0].astype(np.float64) * 2048.0, rtol=1e-12)
+
+
 def test_empty_selection_gives_zero_output_and_neg_inf_lse():
     sh = Sh(n_q_heads=2, n_kv_heads=1, ctx=8, d_qk=4, d_v=4, k_t=3)
     q, K, V, sl = rand_inputs(sh, 11)
