@@ -1,7 +1,7 @@
 """Shared helpers of the GPU parity tests: run the CUDA stages through the C ABI,
 run the oracle on the same seeded inputs, and compare with the rules below.
 
-Comparison rules (north star of this library):
+Comparison rules:
   * block summary and label slab: bit-exact (they are min / max / copies of
     stored values);
   * index sets (blocks, tokens): bit-exact, except swaps at the K-th boundary

@@ -143,7 +143,7 @@ FULL = ["tiny_gqa4k_f32", "gqa48k_bf16", "gqa96k_b8_bf16", "mla64k_b4_bf16"]
 @pytest.mark.parametrize("name", FULL)
 def test_full_size_parity(name):
     res = P().full_stage_parity(W.WORKLOADS[name], name=f"full:{name}")
-    # spec: index sets bit-exact except counted boundary swaps
+    # index sets bit-exact except counted boundary swaps
     assert res["block_swaps"] <= max(1, res["groups"] // 8)
     assert res["token_swaps"] <= max(1, res["groups"] // 8)
 
