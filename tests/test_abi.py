@@ -178,6 +178,21 @@ def test_append_tokens_checks_before_launch(T):
     assert T._lib.tls_append_tokens(ctypes.byref(s), None, None, None, 0, None, None, None, None) == T.TLS_OK
 
 
+def test_binding_refuses_host_tensors_for_device_arguments(T):
+    import torch
+
+    s = good_shape(T)
+    cpu = torch.zeros(16, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        T.tls_block_score_topk(s, cpu, cpu, cpu, cpu)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        T.tls_select_step(s, 256, 256, 256, 256, 256, 256, cpu)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        T.tls_sparse_attn_decode(s, 256, 256, 256, 256, 256, None, ws=cpu)
+    with pytest.raises(ValueError, match="pinned"):
+        T.tls_prefetch_diff(s, 384, cpu, 256, 256, 256, 256, 256, 256, 256)
+
+
 def test_device_error_checks_its_argument(T):
     assert T._lib.tls_device_error(None, 0) == T.TLS_ERR_INVALID_ARG
     assert "flags_out is NULL" in T.tls_last_error()

@@ -114,6 +114,22 @@ def _ptr(x):
     raise TypeError(f"expected a tensor, an int pointer or None, got {type(x)}")
 
 
+def _dptr(x):
+    """Pointer of an argument the kernels read or write on the device: a CUDA
+    tensor (a host tensor is refused here, before it could reach a kernel) or
+    a raw integer pointer, passed as is."""
+    if isinstance(x, torch.Tensor) and x.device.type != "cuda":
+        raise ValueError("expected a CUDA tensor (the kernels address device memory)")
+    return _ptr(x)
+
+
+def _hptr(x):
+    """Pointer of host memory that a kernel reads directly: pinned (page-locked)."""
+    if isinstance(x, torch.Tensor) and x.device.type != "cuda" and not x.is_pinned():
+        raise ValueError("host_kv must be pinned host memory (torch.Tensor.pin_memory())")
+    return _ptr(x)
+
+
 def _stream(stream):
     if stream is None:
         return torch.cuda.current_stream().cuda_stream
@@ -127,7 +143,7 @@ def _ws(ws):
         return None, 0
     if isinstance(ws, tuple):
         return ws
-    return ws.data_ptr(), ws.numel() * ws.element_size()
+    return _dptr(ws), ws.numel() * ws.element_size()
 
 
 def _check(st: int, name: str):
@@ -158,69 +174,69 @@ def tls_slab_bytes(shape: TlsShape) -> int:
 
 
 def tls_build_block_meta(shape, K, seq_lens, label_idx, meta_out, slab_out=None, stream=None):
-    _check(_lib.tls_build_block_meta(ctypes.byref(shape), _ptr(K), _ptr(seq_lens), _ptr(label_idx), _ptr(meta_out),
-                                     _ptr(slab_out), _stream(stream)), "tls_build_block_meta")
+    _check(_lib.tls_build_block_meta(ctypes.byref(shape), _dptr(K), _dptr(seq_lens), _dptr(label_idx), _dptr(meta_out),
+                                     _dptr(slab_out), _stream(stream)), "tls_build_block_meta")
 
 
 def tls_append_tokens(shape, K, old_lens, new_lens, max_append, label_idx, meta_out, slab_out=None, stream=None):
-    _check(_lib.tls_append_tokens(ctypes.byref(shape), _ptr(K), _ptr(old_lens), _ptr(new_lens), int(max_append),
-                                  _ptr(label_idx), _ptr(meta_out), _ptr(slab_out), _stream(stream)),
+    _check(_lib.tls_append_tokens(ctypes.byref(shape), _dptr(K), _dptr(old_lens), _dptr(new_lens), int(max_append),
+                                  _dptr(label_idx), _dptr(meta_out), _dptr(slab_out), _stream(stream)),
            "tls_append_tokens")
 
 
 def tls_block_score_topk(shape, q, meta, seq_lens, block_idx_out, block_score_out=None, ws=None, stream=None):
     wp, wb = _ws(ws)
-    _check(_lib.tls_block_score_topk(ctypes.byref(shape), _ptr(q), _ptr(meta), _ptr(seq_lens), _ptr(block_idx_out),
-                                     _ptr(block_score_out), wp, wb, _stream(stream)), "tls_block_score_topk")
+    _check(_lib.tls_block_score_topk(ctypes.byref(shape), _dptr(q), _dptr(meta), _dptr(seq_lens), _dptr(block_idx_out),
+                                     _dptr(block_score_out), wp, wb, _stream(stream)), "tls_block_score_topk")
 
 
 def tls_token_score_topk(shape, q, slab, label_idx, block_idx, seq_lens, token_idx_out, token_score_out=None,
                          ws=None, stream=None):
     wp, wb = _ws(ws)
-    _check(_lib.tls_token_score_topk(ctypes.byref(shape), _ptr(q), _ptr(slab), _ptr(label_idx), _ptr(block_idx),
-                                     _ptr(seq_lens), _ptr(token_idx_out), _ptr(token_score_out), wp, wb,
+    _check(_lib.tls_token_score_topk(ctypes.byref(shape), _dptr(q), _dptr(slab), _dptr(label_idx), _dptr(block_idx),
+                                     _dptr(seq_lens), _dptr(token_idx_out), _dptr(token_score_out), wp, wb,
                                      _stream(stream)), "tls_token_score_topk")
 
 
 def tls_select_step(shape, q, meta, slab, label_idx, seq_lens, block_idx_out, token_idx_out, block_score_out=None,
                     token_score_out=None, stream=None):
-    _check(_lib.tls_select_step(ctypes.byref(shape), _ptr(q), _ptr(meta), _ptr(slab), _ptr(label_idx),
-                                _ptr(seq_lens), _ptr(block_idx_out), _ptr(token_idx_out), _ptr(block_score_out),
-                                _ptr(token_score_out), _stream(stream)), "tls_select_step")
+    _check(_lib.tls_select_step(ctypes.byref(shape), _dptr(q), _dptr(meta), _dptr(slab), _dptr(label_idx),
+                                _dptr(seq_lens), _dptr(block_idx_out), _dptr(token_idx_out), _dptr(block_score_out),
+                                _dptr(token_score_out), _stream(stream)), "tls_select_step")
 
 
 def tls_sparse_attn_decode(shape, q, K, V, token_idx, out, lse_out=None, ws=None, stream=None):
     wp, wb = _ws(ws)
-    _check(_lib.tls_sparse_attn_decode(ctypes.byref(shape), _ptr(q), _ptr(K), _ptr(V), _ptr(token_idx), _ptr(out),
-                                       _ptr(lse_out), wp, wb, _stream(stream)), "tls_sparse_attn_decode")
+    _check(_lib.tls_sparse_attn_decode(ctypes.byref(shape), _dptr(q), _dptr(K), _dptr(V), _dptr(token_idx), _dptr(out),
+                                       _dptr(lse_out), wp, wb, _stream(stream)), "tls_sparse_attn_decode")
 
 
 def tls_sparse_attn_decode_paged(shape, q, cache, slot_of_block, n_slots, token_idx, out, lse_out=None, ws=None,
                                  stream=None):
     wp, wb = _ws(ws)
-    _check(_lib.tls_sparse_attn_decode_paged(ctypes.byref(shape), _ptr(q), _ptr(cache), _ptr(slot_of_block),
-                                             int(n_slots), _ptr(token_idx), _ptr(out), _ptr(lse_out), wp, wb,
+    _check(_lib.tls_sparse_attn_decode_paged(ctypes.byref(shape), _dptr(q), _dptr(cache), _dptr(slot_of_block),
+                                             int(n_slots), _dptr(token_idx), _dptr(out), _dptr(lse_out), wp, wb,
                                              _stream(stream)), "tls_sparse_attn_decode_paged")
 
 
 def tls_offload_reset(shape, n_slots, slot_of_block, block_of_slot, stream=None):
-    _check(_lib.tls_offload_reset(ctypes.byref(shape), int(n_slots), _ptr(slot_of_block), _ptr(block_of_slot),
+    _check(_lib.tls_offload_reset(ctypes.byref(shape), int(n_slots), _dptr(slot_of_block), _dptr(block_of_slot),
                                   _stream(stream)), "tls_offload_reset")
 
 
 def tls_prefetch_diff(shape, n_slots, host_kv, cache, slot_of_block, block_of_slot, prev_block_idx, next_block_idx,
                       n_new_out, jobs_ws, stream=None):
-    _check(_lib.tls_prefetch_diff(ctypes.byref(shape), int(n_slots), _ptr(host_kv), _ptr(cache), _ptr(slot_of_block),
-                                  _ptr(block_of_slot), _ptr(prev_block_idx), _ptr(next_block_idx), _ptr(n_new_out),
-                                  _ptr(jobs_ws), _stream(stream)), "tls_prefetch_diff")
+    _check(_lib.tls_prefetch_diff(ctypes.byref(shape), int(n_slots), _hptr(host_kv), _dptr(cache), _dptr(slot_of_block),
+                                  _dptr(block_of_slot), _dptr(prev_block_idx), _dptr(next_block_idx), _dptr(n_new_out),
+                                  _dptr(jobs_ws), _stream(stream)), "tls_prefetch_diff")
 
 
 def tls_block_score_topk_noalloc(shape, q, meta, seq_lens, block_idx_out, stream=None):
     """Block selection without a workspace, for callers that cannot allocate
     device memory: the scores live in a fixed array inside the library (see
     include/tls.h for the size limit and the sharing rules)."""
-    _check(_lib.tls_block_score_topk_noalloc(ctypes.byref(shape), _ptr(q), _ptr(meta), _ptr(seq_lens),
-                                             _ptr(block_idx_out), _stream(stream)), "tls_block_score_topk_noalloc")
+    _check(_lib.tls_block_score_topk_noalloc(ctypes.byref(shape), _dptr(q), _dptr(meta), _dptr(seq_lens),
+                                             _dptr(block_idx_out), _stream(stream)), "tls_block_score_topk_noalloc")
 
 
 def tls_wait_event(event, timeout_ms: int) -> int:
