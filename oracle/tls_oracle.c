@@ -21,7 +21,9 @@
  * index, clamping, empty selections) are stated at each function.
  *
  * Inputs are read in their stored type (fp32, or bf16 bits) and widened
- * exactly to double; all arithmetic is double.  Tensor layouts:
+ * exactly to double; all arithmetic is double, except the codes and scales of
+ * the quantised label slab (a variant), which are integers and scales decided
+ * in fp32 (ora_quantize_labels).  Tensor layouts:
  *   q    [B][H_q][d_qk]           K [B][H_kv][max_ctx][d_qk]
  *   V    [B][H_kv][max_ctx][d_v]  (or V = K[..., :d_v] when v_is_k_prefix)
  *   query head h uses KV head h / (H_q / H_kv).
