@@ -41,3 +41,24 @@ def test_two_gloo_ranks_have_independent_work_and_max_time():
     (s0, k0, t0), (s1, k1, t1) = out[0], out[1]
     assert s0 != s1 and k0 != k1
     assert t0 == t1 == 11.0
+
+
+def test_reference_arm_under_torchrun_prints_one_line_from_rank_zero():
+    """`bench.py --impl reference` launched like the multi-GPU bench: rank 0
+    times the oracle and prints the one JSON line; the other rank exits 0
+    without work (no GPU, no process group needed)."""
+    import json
+    import subprocess
+    import sys
+
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), "bench.py", "--impl", "reference",
+           "--gpus", "2", "--steps", "1", "--warmup", "3"]
+    r = subprocess.run(cmd, cwd=root, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout[-3000:]
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
