@@ -150,7 +150,11 @@ TLS_API tls_status tls_build_block_meta(const tls_shape *s, const void *K, const
  *                      a sequence whose range is invalid or longer than
  *                      max_append is left untouched and sets bit 4 of the
  *                      device error word (tls_device_error)
- *   K, label_idx, meta, slab as in tls_build_block_meta. */
+ *   K, label_idx, meta, slab as in tls_build_block_meta.
+ * An int8 label slab (slab_bits 8) is not updated here: a new token can move
+ * a channel's scale and with it every code of the group.  A non-NULL slab
+ * then returns TLS_ERR_UNSUPPORTED; call with slab NULL for the summaries
+ * and rebuild the slab with tls_build_block_meta. */
 TLS_API tls_status tls_append_tokens(const tls_shape *s, const void *K, const int32_t *old_lens,
                                      const int32_t *new_lens, int32_t max_append, const int32_t *label_idx,
                                      void *meta, void *slab, void *stream);
