@@ -1,0 +1,44 @@
+"""Host-side logic of bench.py that the reported numbers rest on (no GPU)."""
+import json
+
+import bench
+from two_level_sparse_quest_b200 import workloads as W
+
+
+def test_algorithmic_bytes_of_the_benchmark_workload():
+    w = W.WORKLOADS["gqa96k_b8_bf16"]
+    ab = bench.algorithmic_bytes(w)
+    G = 8 * 8
+    assert ab["block_summary"] == G * 3072 * 2 * 128 * 2          # every block's max and min rows
+    assert ab["label_slab"] == G * 256 * 32 * 16 * 2              # the K_b * bs candidates' label rows
+    assert ab["gathered_kv"] == G * 4096 * (128 + 128) * 2        # K and V rows of the kept tokens
+    assert ab["total"] == 254084096
+    assert ab["stage_select"] == ab["stage_block"] + ab["stage_token"] - ab["q"]
+    assert sum(ab[k] for k in ("block_summary", "label_slab", "gathered_kv", "q", "out_lse", "indices")) == ab["total"]
+
+
+def test_int8_slab_halves_the_label_bytes_and_adds_the_scales():
+    w = W.WORKLOADS["gqa96k_b8_bf16"]
+    a0 = bench.algorithmic_bytes(w)
+    a8 = bench.algorithmic_bytes(w.with_(slab_bits=8))
+    G = 8 * 8
+    assert a8["label_slab"] == a0["label_slab"] // 2 + G * 16 * 4
+    assert a8["block_summary"] == a0["block_summary"] and a8["gathered_kv"] == a0["gathered_kv"]
+
+
+def test_latent_workload_reads_no_separate_values():
+    w = W.WORKLOADS["mla64k_b4_bf16"]
+    ab = bench.algorithmic_bytes(w)
+    assert ab["gathered_kv"] == 4 * 1 * 2048 * 576 * 2  # V is the first 512 channels of the latent row
+
+
+def test_traffic_is_only_reported_for_the_current_kernel_sources(tmp_path, monkeypatch):
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "abc")
+    (prof / "traffic.json").write_text(json.dumps({"stage_select": {"bytes_per_launch": 5.0, "source_hash": "abc"}}))
+    assert bench.read_traffic("stage_select") == 5.0
+    assert bench.read_traffic("stage_attn") is None
+    (prof / "traffic.json").write_text(json.dumps({"stage_select": {"bytes_per_launch": 5.0, "source_hash": "old"}}))
+    assert bench.read_traffic("stage_select") is None
