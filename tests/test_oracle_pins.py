@@ -87,9 +87,10 @@ def per_head_bounds(sh, q, meta, sl):
     return np.stack(out, axis=1)  # [B][H_q][N_b]
 
 
-@pytest.mark.parametrize("seed", [0, 1, 2])
-def test_block_bound_dominates_every_key(seed):
-    sh = Sh(batch=2, n_q_heads=4, n_kv_heads=2, ctx=40, block_size=8, d_qk=6)
+@pytest.mark.parametrize("seed,heads", [(0, (4, 2)), (1, (4, 2)), (2, (4, 2)), (3, (32, 1)), (4, (1, 1))])
+def test_block_bound_dominates_every_key(seed, heads):
+    # GQA, MQA (32 query heads on one KV head) and MHA (one head per KV head)
+    sh = Sh(batch=2, n_q_heads=heads[0], n_kv_heads=heads[1], ctx=40, block_size=8, d_qk=6)
     q, K, V, sl = rand_inputs(sh, seed, seq_lens=[40, 29])
     s = O.shape_of(sh)
     meta = O.build_meta(s, K, sl)
