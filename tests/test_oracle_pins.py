@@ -470,7 +470,7 @@ def _mutant_lib(tmpdir, name):
 
 
 PIN_FOR_MUTANT = {
-    "bound_uses_min": lambda: test_block_bound_dominates_every_key(0),
+    "bound_uses_min": lambda: test_block_bound_dominates_every_key(0, (4, 2)),
     "bound_drops_min_row": lambda: test_block_bound_is_attained_at_box_corner(),
     "token_score_wrong_channel": lambda: test_token_scores_single_label_channel_is_product(),
     "topk_ties_to_higher": lambda: test_topk_matches_bruteforce_with_ties(0),
