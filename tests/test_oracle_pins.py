@@ -430,6 +430,31 @@ def test_stream_constant_query_has_no_diff_after_first_step():
         np.testing.assert_array_equal(res["out"][t], out)
 
 
+def test_golden_stream_attends_inside_the_previous_selection():
+    """Hand-worked three-step stream whose block selection changes every step:
+    step t must attend inside S_b(t-1) (step 0 inside S_b(0)), so the outputs of
+    steps 1 and 2 differ from attending inside the current or the first selection."""
+    d = _load("stream_lag_three_steps.json")
+    s = _golden_shape(d)
+    qs = np.array(d["q_steps"], np.float32)[:, None, None, :]  # [T][B=1][H_q=1][d]
+    K = np.array(d["K"], np.float32)[None, None]
+    V = np.array(d["V"], np.float32)[None, None]
+    sl = np.array([4], np.int32)
+    L = np.array(d["label_idx"], np.int32)
+    meta = O.build_meta(s, K, sl)
+    res = O.stream_decode(s, qs, K, V, meta, sl, L)
+    e = d["expected"]
+    sig = lambda x: 1.0 / (1.0 + math.exp(-x))
+    want_out = [[sig(1.0), sig(-1.0)], e["out"][1], e["out"][2]]
+    want_lse = [math.log(math.exp(2.0) + math.exp(1.0)), math.log(2.0), math.log(2.0)]
+    for t in range(3):
+        assert res["block_idx"][t][0, 0].tolist() == e["block_idx"][t], f"S_b({t})"
+        assert int(res["n_new"][t][0, 0]) == e["n_new"][t], f"new blocks at step {t}"
+        assert res["token_idx"][t][0, 0].tolist() == e["token_idx"][t], f"tokens at step {t}"
+        np.testing.assert_allclose(res["out"][t][0, 0], want_out[t], rtol=1e-14, atol=1e-15, err_msg=f"step {t}")
+        assert res["lse"][t][0, 0] == pytest.approx(want_lse[t], rel=1e-14)
+
+
 def test_needles_in_kept_blocks_win_token_selection():
     # workload diagnostic, not a parity claim: a planted needle key 4*qbar/|qbar| that sits
     # in a kept block scores far above random keys on the label channels and is kept
@@ -469,7 +494,16 @@ def _mutant_lib(tmpdir, name):
     return so
 
 
+# Mistakes planted in the Python front (oracle.py) rather than the C file.
+PY_MUTANTS = {
+    "stream_attends_in_current": ("attend_in = cur if prev is None else prev", "attend_in = cur"),
+    "stream_attends_in_first": ("attend_in = cur if prev is None else prev",
+                                "attend_in = cur if prev is None else first"),
+}
+
 PIN_FOR_MUTANT = {
+    "stream_attends_in_current": lambda: test_golden_stream_attends_inside_the_previous_selection(),
+    "stream_attends_in_first": lambda: test_golden_stream_attends_inside_the_previous_selection(),
     "bound_uses_min": lambda: test_block_bound_dominates_every_key(0, (4, 2)),
     "bound_drops_min_row": lambda: test_block_bound_is_attained_at_box_corner(),
     "token_score_wrong_channel": lambda: test_token_scores_single_label_channel_is_product(),
@@ -477,6 +511,32 @@ PIN_FOR_MUTANT = {
     "softmax_drops_scale": lambda: test_full_selection_equals_full_attention(W.F32),
     "meta_min_is_max": lambda: test_meta_equals_bruteforce_minmax(W.F32),
 }
+
+
+def _py_mutant_module(name):
+    """A copy of oracle.py with one planted mistake, loaded as its own module
+    (it loads the same, unmodified liboracle.so)."""
+    import types
+
+    src = open(O.__file__).read()
+    old, new = PY_MUTANTS[name]
+    assert src.count(old) == 1, name
+    if name == "stream_attends_in_first":  # also remember the first selection
+        src = src.replace("    prev = None\n", "    prev = None\n    first = None\n", 1)
+        src = src.replace("        prev = cur\n", "        prev = cur\n        first = cur if first is None else first\n", 1)
+    mod = types.ModuleType(f"oracle_mutant_{name}")
+    mod.__file__ = O.__file__
+    exec(compile(src.replace(old, new), f"oracle_mutant_{name}.py", "exec"), mod.__dict__)
+    mod.lib, mod.OraShape = O.lib, O.OraShape  # the loaded library and its argument types
+    return mod
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTANTS))
+def test_planted_python_mistake_is_caught(name, monkeypatch):
+    mod = _py_mutant_module(name)
+    monkeypatch.setattr(O, "stream_decode", mod.stream_decode)
+    with pytest.raises(AssertionError):
+        PIN_FOR_MUTANT[name]()
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
