@@ -31,8 +31,13 @@ SWAP_RTOL = 1e-4
 
 REPORT = os.environ.get("TLS_PARITY_REPORT")
 
+# Every parity case's swap counts, printed at the end of the pytest session
+# (tests/conftest.py) so that they appear in the run's output.
+RESULTS: list = []
+
 
 def report(name: str, **kv):
+    RESULTS.append({"case": name, **kv})
     if not REPORT:
         return
     os.makedirs(os.path.dirname(REPORT) or ".", exist_ok=True)
@@ -293,6 +298,36 @@ def full_stage_parity(w: W.Workload, seq_lens=None, out_dtype=0, name=None, inp=
     out, lse = gpu.attention(to_dev(orc.token_idx))
     torch.cuda.synchronize()
     err = check_attention(gpu.out_f64(out), lse.cpu().numpy().astype(np.float64), orc.out, orc.lse, f"{name} attention")
+    # stages 1-4 in one launch (tls_select_step, the call the benchmark times)
+    # against the oracle: block ids directly; token ids wherever the launch's
+    # own block selection equals the oracle's (elsewhere the candidates differ
+    # by a counted block swap and only the self-consistency of the kernel's
+    # token ranking on its own fp32 scores is checked)
+    fb = torch.full((w.batch, w.n_kv_heads, w.k_b), -7, dtype=torch.int32, device="cuda")
+    ft = torch.full((w.batch, w.n_kv_heads, w.k_t), -7, dtype=torch.int32, device="cuda")
+    fbs = torch.zeros((w.batch, w.n_kv_heads, w.n_blocks), dtype=torch.float32, device="cuda")
+    fts = torch.zeros((w.batch, w.n_kv_heads, w.k_b * w.block_size), dtype=torch.float32, device="cuda")
+    tls().tls_select_step(gpu.shape, gpu.q, gpu.meta, gpu.slab, gpu.label, gpu.seq_lens, fb, ft, fbs, fts)
+    torch.cuda.synchronize()
+    fb, ft, fbs, fts = fb.cpu().numpy(), ft.cpu().numpy(), fbs.cpu().numpy(), fts.cpu().numpy()
+    check_scores(fbs, orc.block_scores, block_score_bound(w, inp, orc), f"{name} select_step block scores")
+    step_swaps_b = step_swaps_t = 0
+    C = w.k_b * w.block_size
+    for b in range(w.batch):
+        nb = -(-int(inp.seq_lens[b]) // w.block_size)
+        ids = np.arange(nb, dtype=np.int32)
+        for g in range(w.n_kv_heads):
+            what = f"{name} select_step b{b} g{g}"
+            step_swaps_b += check_selection(fb[b, g], ids, orc.block_scores[b, g, :nb], w.k_b, what + " blocks")
+            j = np.arange(C)
+            blk = fb[b, g][j // w.block_size]
+            cand = np.where(blk >= 0, blk * w.block_size + j % w.block_size, -1)
+            ok = (cand >= 0) & (cand < inp.seq_lens[b])
+            if (fb[b, g] == orc.block_idx[b, g]).all():
+                oko = orc.cand_tok[b, g] >= 0
+                step_swaps_t += check_selection(ft[b, g], orc.cand_tok[b, g][oko], orc.cand_scores[b, g][oko], w.k_t,
+                                                what + " tokens")
+            check_selection_self_consistent(ft[b, g], cand[ok].astype(np.int32), fts[b, g][ok], what + " tokens")
     # chained: the GPU's own selections all the way
     cb, _ = gpu.block_stage(with_scores=False)
     ct, _ = gpu.token_stage(cb, with_scores=False)
@@ -312,7 +347,8 @@ def full_stage_parity(w: W.Workload, seq_lens=None, out_dtype=0, name=None, inp=
                 hs = slice(g * G, (g + 1) * G)
                 check_attention(cout[b, hs], clse[b, hs], orc.out[b, hs], orc.lse[b, hs], f"{name} chained b{b} g{g}")
     assert tls().tls_device_error(clear=True) == 0, f"{name}: a kernel's bounded wait gave up"
-    res = dict(block_swaps=swaps_b, token_swaps=swaps_t, attn_max_abs_err=err,
+    res = dict(block_swaps=swaps_b, token_swaps=swaps_t, step_block_swaps=step_swaps_b,
+               step_token_swaps=step_swaps_t, attn_max_abs_err=err,
                chained_groups_identical=same_groups, groups=w.batch * w.n_kv_heads)
     report(name, **res)
     return res
