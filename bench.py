@@ -26,11 +26,14 @@ import sys
 import threading
 import time
 
+import numpy as np
+
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "sparse-attn decode steps/sec (all heads) at 96k ctx; achieved HBM GB/s vs peak"
 N_LAYERS_DEFAULT = 4
+STAGE_STEPS_MIN = 100  # steps of the separate per-stage timing pass
 SMI_FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -83,9 +86,9 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def read_traffic(stage: str):
-    """DRAM traffic per launch from a committed ncu summary, only if it was
-    taken on the kernel sources as they are now."""
+def read_profile(stage: str):
+    """The committed ncu summary entry of a stage (profiles/traffic.json), only
+    if it was taken on the kernel sources as they are now."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -94,7 +97,14 @@ def read_traffic(stage: str):
     ent = d.get(stage)
     if not ent or ent.get("source_hash") != kernel_source_hash():
         return None
-    return ent.get("bytes_per_launch")
+    return ent
+
+
+def read_traffic(stage: str):
+    """DRAM traffic per launch from a committed ncu summary (null when the
+    kernels changed since the counters were taken)."""
+    ent = read_profile(stage)
+    return ent.get("bytes_per_launch") if ent else None
 
 
 class ClockSampler:
@@ -216,7 +226,6 @@ def gpu_arm(args, rank, world, local_rank):
 
     K0 = up(inp.K)
     V0 = up(inp.V) if inp.V is not None else None
-    del inp.K
     seq_lens, label = up(inp.seq_lens), up(inp.label_idx)
     layers = [Layer(T, w, shape, K0, V0, seq_lens, label, up(qs[i]), dev) for i in range(N_LAYERS)]
     del K0, V0
@@ -245,11 +254,8 @@ def gpu_arm(args, rank, world, local_rank):
         step(layers[i % N_LAYERS])
     torch.cuda.synchronize()
 
-    # ---- timed region: K steps.  Kernels within and across stages are chained by
-    # programmatic dependent launch; per-stage CUDA events (which break that
-    # overlap at the stage boundaries) are recorded on every SAMPLE-th step only.
-    SAMPLE = 32
-    evs = {i: [torch.cuda.Event(enable_timing=True) for _ in range(3)] for i in range(0, args.steps, SAMPLE)}
+    # ---- timed region: exactly K steps, nothing else on the stream.  Kernels
+    # within and across steps are chained by programmatic dependent launch.
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
@@ -262,7 +268,7 @@ def gpu_arm(args, rank, world, local_rank):
     sampler.mark("t0")
     t_start.record(stream)
     for i in range(args.steps):
-        step(layers[i % N_LAYERS], evs.get(i))
+        step(layers[i % N_LAYERS])
     t_end.record(stream)
     torch.cuda.synchronize()
     sampler.mark("t1")
@@ -270,9 +276,20 @@ def gpu_arm(args, rank, world, local_rank):
         dist.barrier()
     clocks = sampler.stop() if rank == 0 else None
     ms = t_start.elapsed_time(t_end)
-    st = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2])] for e in evs.values()])
-    stage_ms = st.mean(axis=0)
     ms = max_over_ranks(ms, dev)
+
+    # ---- per-stage times, in a separate untimed pass: CUDA events around each
+    # C call on every step (the events cut the launch chain at the stage
+    # boundaries, which is why they stay out of the timed region).  The first
+    # step of the pass is dropped.
+    n_stage = max(STAGE_STEPS_MIN, min(args.steps, 1000))
+    sev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_stage + 1)]
+    for i in range(n_stage + 1):
+        step(layers[i % N_LAYERS], sev[i])
+    torch.cuda.synchronize()
+    st = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2])] for e in sev[1:]])
+    stage_ms = st.mean(axis=0)
+    stage_med = np.median(st, axis=0)
 
     # ---- end to end through the C ABI with host buffers: every step uploads its
     # q from pinned host memory and reads its out + lse back.  The copies run on
@@ -332,7 +349,7 @@ def gpu_arm(args, rank, world, local_rank):
     d2h = out.numel() * out.element_size() + lse.numel() * lse.element_size()
 
     if rank != 0:
-        return None
+        return None, None
     ab = algorithmic_bytes(w)
     peaks = read_peaks()
     step_ms = ms / args.steps
@@ -340,6 +357,13 @@ def gpu_arm(args, rank, world, local_rank):
     dom = int(np.argmax(stage_ms))
     dom_bytes = ab[names[dom]]
     achieved = dom_bytes / (stage_ms[dom] * 1e-3) / 1e9
+    # a stage inside the step cannot take longer than the whole step; if the
+    # separately timed stage does (it runs without the launch chain), say so
+    consistent = bool(stage_ms[dom] <= step_ms * 1.05)
+    if not consistent:
+        print(f"warning: {names[dom]} mean {stage_ms[dom] * 1e3:.1f} us > step {step_ms * 1e3:.1f} us",
+              file=sys.stderr)
+    prof = read_profile(names[dom])
     res = {
         "metric": METRIC,
         "value": world * args.steps / (ms * 1e-3),
@@ -365,18 +389,29 @@ def gpu_arm(args, rank, world, local_rank):
         "hbm_frac_of_measured": ab["total"] / (step_ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
         "hbm_frac_of_8000": ab["total"] / (step_ms * 1e-3) / 1e9 / 8000.0,
         "stages_us": {n: float(v * 1e3) for n, v in zip(names, stage_ms)},
-        "stage_timing": f"CUDA events around each stage call on every {SAMPLE}th step of the timed region",
+        "stages_median_us": {n: float(v * 1e3) for n, v in zip(names, stage_med)},
+        "stage_timing": f"separate untimed pass of {n_stage} steps after the timed region, CUDA events around "
+                        f"each stage call on every step (first step dropped); mean reported",
         "roofline": {
             "kernel": names[dom], "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],
             "traffic": read_traffic(names[dom]), "algorithmic_bytes_per_launch": dom_bytes,
+            "stage_us": float(stage_ms[dom] * 1e3), "samples": n_stage,
+            "consistent_with_step": consistent,
+            "cross_check": {
+                "whole_step_gbs": ab["total"] / (step_ms * 1e-3) / 1e9,
+                "profile_mean_us": prof.get("mean_us") if prof else None,
+                "profile_frac": (dom_bytes / (prof["mean_us"] * 1e-6) / 1e9 / peaks["hbm_gbs"]
+                                 if prof and prof.get("mean_us") else None),
+                "profile_source": prof.get("capture") if prof else None,
+            },
         },
         "e2e": {"value": world * n_e2e / (e2e_ms * 1e-3), "unit": "steps/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": n_e2e},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
-    return res
+    return res, inp
 
 
 # ----------------------------------------------------------------------------- offload stream
@@ -526,52 +561,127 @@ def dense_arm(args):
 
 
 # ----------------------------------------------------------------------------- CPU oracle
-def oracle_sample(args, budget_s: float):
-    """The fp64 oracle (single thread) on a bounded sample of the workload: the
-    step for a subset of the batch rows, scaled to a whole step."""
-    import numpy as np
+class OracleStep:
+    """The fp64 oracle's decode step (stages 1-5 from the block summary on) on
+    the host cores.  The step's (sequence, KV head) groups are independent, so
+    each is its own oracle call on a one-group shape; a thread pool runs them
+    concurrently (the oracle is C called through ctypes, which releases the
+    GIL for the duration of each call).  The block summaries are built once,
+    untimed, as the GPU side builds them once per KV cache."""
 
-    from oracle import oracle as O
-    from two_level_sparse_quest_b200 import workloads as W
+    def __init__(self, w, inp, threads: int):
+        from concurrent.futures import ThreadPoolExecutor
 
-    w = W.WORKLOADS[args.workload]
-    rows = 1
-    ws = w.with_(batch=rows)
-    inp = W.make_decode_inputs(ws)
-    s = O.shape_of(ws)
-    meta = O.build_meta(s, inp.K, inp.seq_lens)
+        from oracle import oracle as O
+
+        self.O, self.w, self.threads = O, w, threads
+        G = w.group
+        self.s = O.shape_of(w.with_(batch=1, n_kv_heads=1, n_q_heads=G))
+        self.groups = []
+        for b in range(w.batch):
+            for g in range(w.n_kv_heads):
+                self.groups.append(dict(
+                    q=inp.q[b:b + 1, g * G:(g + 1) * G], K=inp.K[b:b + 1, g:g + 1],
+                    V=None if inp.V is None else inp.V[b:b + 1, g:g + 1],
+                    sl=inp.seq_lens[b:b + 1], label=inp.label_idx))
+        self.pool = ThreadPoolExecutor(max_workers=threads)
+
+        def meta(gr):
+            gr["meta"] = O.build_meta(self.s, gr["K"], gr["sl"])
+
+        list(self.pool.map(meta, self.groups))
+
+    def _one(self, gr):
+        self.O.decode_step(self.s, np.ascontiguousarray(gr["q"]), gr["K"], gr["V"], gr["meta"], gr["sl"], gr["label"])
+
+    def run(self, n_groups=None, threads=True) -> float:
+        """Seconds for the first n_groups groups (all by default), on the pool
+        or on this thread alone."""
+        todo = self.groups[:n_groups] if n_groups else self.groups
+        t0 = time.perf_counter()
+        if threads:
+            list(self.pool.map(self._one, todo))
+        else:
+            for gr in todo:
+                self._one(gr)
+        return time.perf_counter() - t0
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def oracle_baseline(w, inp, budget_s: float) -> dict:
+    """The oracle timed on all host cores on whole decode steps of the
+    workload (a bounded number of them), plus one single-thread figure."""
+    cores = host_cores()
+    os_ = OracleStep(w, inp, cores)
+    n_groups = len(os_.groups)
+    # single thread: a few groups, scaled to the step (the groups are alike)
+    k1 = max(1, min(n_groups, 4))
+    t1 = os_.run(k1, threads=False) * n_groups / k1
     times = []
     t_all = time.time()
     while True:
-        t0 = time.perf_counter()
-        O.decode_step(s, inp.q, inp.K, inp.V, meta, inp.seq_lens, inp.label_idx)
-        times.append(time.perf_counter() - t0)
-        if time.time() - t_all > budget_s or len(times) >= 20:
+        times.append(os_.run())
+        if time.time() - t_all > budget_s or len(times) >= 10:
             break
-    per_row = float(np.median(times)) / rows
-    per_step = per_row * w.batch
+    per_step = float(np.median(times))
     return {
-        "value": 1.0 / per_step, "unit": "steps/s", "cores": 1, "kind": "oracle",
-        "sample": f"{len(times)} run(s) of {rows} of {w.batch} batch rows (all {w.n_kv_heads} KV heads), "
-                  f"stages 1-5, fp64, single thread; scaled x{w.batch // rows} to one step",
+        "value": 1.0 / per_step, "unit": "steps/s", "cores": cores, "kind": "oracle",
+        "sample": f"{len(times)} whole decode step(s) of {args_workload_name(w)} (all {n_groups} (sequence, KV head) "
+                  f"groups, stages 1-5 from the block summary), fp64, {cores} threads over the groups; median",
         "seconds_per_step": per_step,
+        "single_thread": {"value": 1.0 / t1, "unit": "steps/s", "seconds_per_step": t1,
+                          "sample": f"{k1} of {n_groups} groups on one thread, scaled x{n_groups / k1:g}"},
     }
 
 
+def args_workload_name(w) -> str:
+    return getattr(w, "name", "workload")
+
+
 def reference_arm(args, rank, world):
+    """The oracle as the reference arm: --warmup untimed and --steps timed
+    decode steps of the workload on all host cores (rank 0 only).  When a
+    whole step would not let the run end within a few minutes, each step is a
+    fixed sample of the step's groups, scaled, and the line says so."""
     if rank != 0:
         return None
     from two_level_sparse_quest_b200 import workloads as W
 
     w = W.WORKLOADS[args.workload]
-    # warm-up and timed steps are each a bounded sample (one batch row)
-    cb = oracle_sample(args, budget_s=max(5.0, 3.0 * (args.steps + args.warmup)))
+    inp = W.make_decode_inputs(w)
+    cores = host_cores()
+    os_ = OracleStep(w, inp, cores)
+    n_groups = len(os_.groups)
+    probe = os_.run(min(n_groups, cores))  # one round of the pool
+    est_step = probe * math.ceil(n_groups / cores) if n_groups > cores else probe
+    budget = 150.0
+    n_sample = n_groups
+    if est_step * (args.steps + args.warmup) > budget:
+        n_sample = max(1, min(n_groups, int(n_groups * budget / (est_step * (args.steps + args.warmup)))))
+    for _ in range(args.warmup):
+        os_.run(n_sample)
+    times = [os_.run(n_sample) * n_groups / n_sample for _ in range(args.steps)]
+    total = float(np.sum(times))
+    per_step = total / args.steps
+    sample = (f"every step is the whole decode step ({n_groups} groups)" if n_sample == n_groups
+              else f"every step runs {n_sample} of {n_groups} groups, scaled x{n_groups / n_sample:g}")
+    cb = {"value": 1.0 / per_step, "unit": "steps/s", "cores": cores, "kind": "oracle",
+          "sample": f"{args.warmup} warm-up + {args.steps} timed steps; {sample}; fp64, {cores} threads over the groups",
+          "seconds_per_step": per_step}
     return {
         "metric": METRIC, "impl": "reference", "value": cb["value"], "unit": "steps/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": cb["seconds_per_step"] * 1e3,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic: seeded Gaussian K/V with outlier channels and planted needle keys",
-        "config": {"workload": args.workload, "batch": w.batch, "ctx": w.ctx, "k_b": w.k_b, "k_t": w.k_t},
+        "config": {"workload": args.workload, "batch": w.batch, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
+                   "d_qk": w.d_qk, "d_v": w.d_v, "ctx": w.ctx, "block_size": w.block_size, "k_b": w.k_b,
+                   "k_t": w.k_t, "n_label": w.n_label},
         "cpu_baseline": cb,
         "e2e": {"value": cb["value"], "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "note": "reference arm = the fp64 CPU oracle (no runnable reference implementation exists)",
@@ -625,10 +735,12 @@ def main():
         import torch.distributed as dist
 
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    res = gpu_arm(args, rank, world, local_rank)
+    res, inp = gpu_arm(args, rank, world, local_rank)
     if rank == 0 and res is not None:
         if world == 1 and not args.no_cpu_baseline:
-            res["cpu_baseline"] = oracle_sample(args, budget_s=15.0)
+            from two_level_sparse_quest_b200 import workloads as W
+
+            res["cpu_baseline"] = oracle_baseline(W.WORKLOADS[args.workload], inp, budget_s=15.0)
         print(json.dumps(res), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -42,3 +42,30 @@ def test_traffic_is_only_reported_for_the_current_kernel_sources(tmp_path, monke
     assert bench.read_traffic("stage_attn") is None
     (prof / "traffic.json").write_text(json.dumps({"stage_select": {"bytes_per_launch": 5.0, "source_hash": "old"}}))
     assert bench.read_traffic("stage_select") is None
+
+
+def test_oracle_baseline_splits_the_step_into_its_groups_without_changing_it():
+    """The CPU baseline runs each (sequence, KV head) group as its own oracle
+    call on a thread pool; that must be the same computation as the oracle on
+    the whole batch."""
+    import numpy as np
+
+    from oracle import oracle as O
+
+    w = W.WORKLOADS["gqa48k_bf16"].with_(batch=2, n_kv_heads=2, n_q_heads=8, ctx=1024, k_b=8, k_t=64)
+    inp = W.make_decode_inputs(w, seq_lens=[1024, 777])
+    st = bench.OracleStep(w, inp, threads=3)
+    assert len(st.groups) == 4
+    s = O.shape_of(w)
+    meta = O.build_meta(s, inp.K, inp.seq_lens)
+    bidx, tidx, out, lse = O.decode_step(s, inp.q, inp.K, inp.V, meta, inp.seq_lens, inp.label_idx)
+    G = w.group
+    for i, gr in enumerate(st.groups):
+        b, g = divmod(i, w.n_kv_heads)
+        rb, rt, ro, rl = O.decode_step(st.s, np.ascontiguousarray(gr["q"]), gr["K"], gr["V"], gr["meta"], gr["sl"],
+                                       gr["label"])
+        np.testing.assert_array_equal(rb[0, 0], bidx[b, g])
+        np.testing.assert_array_equal(rt[0, 0], tidx[b, g])
+        np.testing.assert_array_equal(ro[0], out[b, g * G:(g + 1) * G])
+        np.testing.assert_array_equal(rl[0], lse[b, g * G:(g + 1) * G])
+    assert st.run() > 0 and st.run(2, threads=False) > 0
