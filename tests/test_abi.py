@@ -97,6 +97,9 @@ def test_version_and_last_error(T):
     (dict(k_b=1025, block_size=8), "TLS_ERR_UNSUPPORTED"),
     (dict(k_b=600), "TLS_ERR_UNSUPPORTED"),          # 600 * 32 candidates > 16384
     (dict(max_ctx=1 << 20, block_size=32), "TLS_ERR_UNSUPPORTED"),
+    # ceil(max_ctx / bs) must not wrap in int: near INT32_MAX it is refused, never a negative count
+    (dict(max_ctx=2 ** 31 - 1, block_size=1 << 20), "TLS_ERR_UNSUPPORTED"),
+    (dict(max_ctx=2 ** 31 - 16, block_size=32), "TLS_ERR_UNSUPPORTED"),
     (dict(v_is_k_prefix=True, n_q_heads=64, n_kv_heads=1, d_qk=576, d_v=512, kv_dtype=0), "TLS_ERR_UNSUPPORTED"),
 ])
 def test_shape_checks_return_status(T, kw, status):

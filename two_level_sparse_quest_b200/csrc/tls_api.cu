@@ -39,7 +39,11 @@ tls_status cuda_status(cudaError_t e, const char *what) {
 
 bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-int n_blocks_max(const tls_shape *s) { return (s->max_ctx + s->block_size - 1) / s->block_size; }
+// ceil(max_ctx / block_size) in 64-bit (max_ctx near INT_MAX must not wrap);
+// max_ctx <= INT_MAX keeps the quotient in int range.
+int n_blocks_max(const tls_shape *s) {
+  return static_cast<int>((static_cast<long long>(s->max_ctx) + s->block_size - 1) / s->block_size);
+}
 
 int device_sms() {
   static int cache[64] = {};
@@ -64,6 +68,9 @@ tls_status check_shape(const tls_shape *s) {
   if (s->out_dtype != TLS_F32 && s->out_dtype != TLS_BF16) return fail(TLS_ERR_INVALID_ARG, "out_dtype %d", s->out_dtype);
   if (s->block_size < 1) return fail(TLS_ERR_INVALID_ARG, "block_size < 1");
   if (s->max_ctx < 1) return fail(TLS_ERR_INVALID_ARG, "max_ctx < 1");
+  // kernels form seq_len + block_size - 1 in int
+  if (s->max_ctx > INT32_MAX - s->block_size)
+    return fail(TLS_ERR_UNSUPPORTED, "max_ctx + block_size exceeds the int32 range");
   if (s->k_b < 1 || s->k_t < 1) return fail(TLS_ERR_INVALID_ARG, "k_b and k_t must be >= 1");
   if (s->d_qk < 1 || s->d_v < 1) return fail(TLS_ERR_INVALID_ARG, "d_qk and d_v must be >= 1");
   if (s->v_is_k_prefix && s->d_v > s->d_qk) return fail(TLS_ERR_INVALID_ARG, "v_is_k_prefix needs d_v <= d_qk");
