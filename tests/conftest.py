@@ -17,6 +17,7 @@ def pytest_terminal_summary(terminalreporter, exitstatus, config):
     the two oracle scores lie within 1e-4 relative (counted, not hidden)."""
     mod = sys.modules.get("tests._parity")
     rows = getattr(mod, "RESULTS", None) if mod else None
+    rows = [r for r in (rows or []) if "block_swaps" in r]
     if not rows:
         return
     tr = terminalreporter
