@@ -285,6 +285,16 @@ TLS_API tls_status tls_prefetch_diff(const tls_shape *s, int32_t n_slots, const 
 TLS_API tls_status tls_block_score_topk_noalloc(const tls_shape *s, const void *q, const void *meta,
                                                 const int32_t *seq_lens, int32_t *block_idx_out, void *stream);
 
+/* Copies the first `count` fp32 block scores that the last
+ * tls_block_score_topk_noalloc call on the current device left in the
+ * library's built-in array into dst (device or pinned host memory; layout
+ * [B][H_kv][ceil(max_ctx/bs)] of that call's shape), asynchronously on
+ * `stream`.  Order it after that call (same stream, or an event).  It is how
+ * such a caller, which has no block_score_out buffer of its own to pass,
+ * reads the scores back; it allocates nothing.
+ * count > 1048576 returns TLS_ERR_INVALID_ARG. */
+TLS_API tls_status tls_noalloc_read_scores(float *dst, size_t count, void *stream);
+
 /* Device-side failure flags of the current device.  Kernels that wait on
  * other CTAs or on the tensor-core/copy engines bound every wait; when one
  * gives up (which a correct run never sees) the kernel still ends, its outputs

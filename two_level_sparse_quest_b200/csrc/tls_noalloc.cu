@@ -79,4 +79,20 @@ tls_status tls_block_score_topk_noalloc(const tls_shape *s, const void *q, const
   return tls_block_score_topk(s, q, meta, seq_lens, block_idx_out, nullptr, nullptr, 0, stream);
 }
 
+tls_status tls_noalloc_read_scores(float *dst, size_t count, void *stream) {
+  if (count == 0) return TLS_OK;
+  if (!dst) return tls::set_error(TLS_ERR_INVALID_ARG, "dst is NULL");
+  if (count > kNoAllocMaxScores)
+    return tls::set_error(TLS_ERR_INVALID_ARG, "count %zu exceeds the built-in array (%zu scores)", count,
+                          kNoAllocMaxScores);
+  float *scores = nullptr;
+  tls_status st = scratch_for_current_device(&scores);
+  if (st != TLS_OK) return st;
+  cudaError_t e = cudaMemcpyAsync(dst, scores, count * sizeof(float), cudaMemcpyDefault,
+                                  static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess)
+    return tls::set_error(TLS_ERR_CUDA, "copying the built-in score array: %s", cudaGetErrorString(e));
+  return TLS_OK;
+}
+
 }  // extern "C"

@@ -31,7 +31,7 @@ STATUS_NAMES = {0: "TLS_OK", 1: "TLS_ERR_INVALID_ARG", 2: "TLS_ERR_UNSUPPORTED",
 EXPORTED = ("tls_version", "tls_last_error", "tls_workspace_size", "tls_build_block_meta", "tls_block_score_topk",
             "tls_token_score_topk", "tls_sparse_attn_decode", "tls_sparse_attn_decode_paged", "tls_offload_reset",
             "tls_prefetch_diff", "tls_wait_event", "tls_block_score_topk_noalloc", "tls_device_error", "tls_select_step",
-            "tls_append_tokens", "tls_slab_bytes")
+            "tls_append_tokens", "tls_slab_bytes", "tls_noalloc_read_scores")
 
 
 class TlsShape(ctypes.Structure):
@@ -72,6 +72,7 @@ _sigs = {
     "tls_select_step": ([_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "tls_append_tokens": ([_S, _P, _P, _P, _i32, _P, _P, _P, _P], ctypes.c_int),
     "tls_slab_bytes": ([_S], _sz),
+    "tls_noalloc_read_scores": ([_P, _sz, _P], ctypes.c_int),
 }
 for _name, (_args, _ret) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -237,6 +238,12 @@ def tls_block_score_topk_noalloc(shape, q, meta, seq_lens, block_idx_out, stream
     include/tls.h for the size limit and the sharing rules)."""
     _check(_lib.tls_block_score_topk_noalloc(ctypes.byref(shape), _dptr(q), _dptr(meta), _dptr(seq_lens),
                                              _dptr(block_idx_out), _stream(stream)), "tls_block_score_topk_noalloc")
+
+
+def tls_noalloc_read_scores(dst, count: int, stream=None):
+    """Copies the first `count` block scores that the last
+    tls_block_score_topk_noalloc call left in the library's array into dst."""
+    _check(_lib.tls_noalloc_read_scores(_dptr(dst), int(count), _stream(stream)), "tls_noalloc_read_scores")
 
 
 def tls_wait_event(event, timeout_ms: int) -> int:
