@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "sparse-attn decode steps/sec (all heads) at 96k ctx; achieved HBM GB/s vs peak"
 N_LAYERS_DEFAULT = 4
+L2_BYTES = 126e6
 STAGE_STEPS_MIN = 100  # steps of the separate per-stage timing pass
 SMI_FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -218,7 +219,9 @@ def gpu_arm(args, rank, world, local_rank):
     w = rank_workload(base, rank)
     shape = T.shape_from_workload(w)
     inp = W.make_decode_inputs(w)
-    N_LAYERS = args.layers
+    # layer copies rotated through: enough that one rotation's algorithmic bytes
+    # are at least twice the 126 MB L2, so no step finds its data in L2
+    N_LAYERS = args.layers or max(N_LAYERS_DEFAULT, math.ceil(2 * L2_BYTES / algorithmic_bytes(w)["total"]))
     qs = W.make_query_stream(w.with_(ar_rho=0.5), steps=N_LAYERS)
 
     def up(a):
@@ -703,8 +706,8 @@ def main():
                     help="time the offload engine on the streaming workload instead (one JSON line of its own)")
     ap.add_argument("--slab-bits", type=int, default=0, choices=[0, 8],
                     help="label slab storage: 0 = the K dtype (the method), 8 = int8 codes + per-channel scales")
-    ap.add_argument("--layers", type=int, default=N_LAYERS_DEFAULT,
-                    help="layer copies rotated through (4 keeps the per-rotation working set above L2)")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="layer copies rotated through (default: enough for twice the L2 per rotation, at least 4)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
