@@ -242,14 +242,17 @@ def gpu_arm(args, rank, world, local_rank):
     sh = stream.cuda_stream
 
     def step(L, ev=None):
-        if ev:
-            ev[0].record(stream)
+        """One decode step through the public call, tls_decode_step."""
+        T.tls_decode_step(shape, L.q, L.meta, L.slab, label, seq_lens, L.K, L.V, bidx, tidx, out, lse, None, None,
+                          ws, sh)
+
+    def step_stages(L, ev):
+        """The same step as its two calls, with CUDA events around each."""
+        ev[0].record(stream)
         T.tls_select_step(shape, L.q, L.meta, L.slab, label, seq_lens, bidx, tidx, None, None, sh)
-        if ev:
-            ev[1].record(stream)
+        ev[1].record(stream)
         T.tls_sparse_attn_decode(shape, L.q, L.K, L.V, tidx, out, lse, ws, sh)
-        if ev:
-            ev[2].record(stream)
+        ev[2].record(stream)
 
     # stages 1-4 (one cluster launch), attention split, log-sum-exp merge
     launches_per_step = 3
@@ -288,9 +291,10 @@ def gpu_arm(args, rank, world, local_rank):
     n_stage = max(STAGE_STEPS_MIN, min(args.steps, 1000))
     sev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_stage + 1)]
     for i in range(n_stage + 1):
-        step(layers[i % N_LAYERS], sev[i])
+        step_stages(layers[i % N_LAYERS], sev[i])
     torch.cuda.synchronize()
     st = np.array([[e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2])] for e in sev[1:]])
+    names = ["stage_select", "stage_attn"]
     stage_ms = st.mean(axis=0)
     stage_med = np.median(st, axis=0)
 
@@ -323,8 +327,8 @@ def gpu_arm(args, rank, world, local_rank):
         stream.wait_event(ev_up[j])
         if i >= 2:
             stream.wait_event(ev_down[j])  # od[j], ld[j] are no longer read
-        T.tls_select_step(shape, qd[j], L.meta, L.slab, label, seq_lens, bidx, tidx, None, None, sh)
-        T.tls_sparse_attn_decode(shape, qd[j], L.K, L.V, tidx, od[j], ld[j], ws, sh)
+        T.tls_decode_step(shape, qd[j], L.meta, L.slab, label, seq_lens, L.K, L.V, bidx, tidx, od[j], ld[j], None,
+                          None, ws, sh)
         ev_comp[j].record(stream)
         down_s.wait_event(ev_comp[j])
         with torch.cuda.stream(down_s):
@@ -356,8 +360,7 @@ def gpu_arm(args, rank, world, local_rank):
     ab = algorithmic_bytes(w)
     peaks = read_peaks()
     step_ms = ms / args.steps
-    names = ["stage_select", "stage_attn"]
-    dom = int(np.argmax(stage_ms))
+    dom = int(np.argmax(stage_ms))  # the roofline's stage: the slower of the two calls
     dom_bytes = ab[names[dom]]
     achieved = dom_bytes / (stage_ms[dom] * 1e-3) / 1e9
     # a stage inside the step cannot take longer than the whole step; if the
@@ -393,8 +396,10 @@ def gpu_arm(args, rank, world, local_rank):
         "hbm_frac_of_8000": ab["total"] / (step_ms * 1e-3) / 1e9 / 8000.0,
         "stages_us": {n: float(v * 1e3) for n, v in zip(names, stage_ms)},
         "stages_median_us": {n: float(v * 1e3) for n, v in zip(names, stage_med)},
-        "stage_timing": f"separate untimed pass of {n_stage} steps after the timed region, CUDA events around "
-                        f"each stage call on every step (first step dropped); mean reported",
+        "stage_timing": f"separate untimed pass of {n_stage} steps after the timed region: the step as its two "
+                        f"calls (tls_select_step, tls_sparse_attn_decode), CUDA events around each on every step "
+                        f"(first step dropped); mean reported",
+        "step_call": "tls_decode_step",
         "roofline": {
             "kernel": names[dom], "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
             "frac": achieved / peaks["hbm_gbs"], "peak_source": peaks["source"],

@@ -105,8 +105,9 @@ TLS_API const char *tls_version(void);
 /* Message of the last failed call on this thread ("" if none). */
 TLS_API const char *tls_last_error(void);
 
-/* Bytes of device workspace that tls_sparse_attn_decode(_paged) need for this
- * shape on the current device (the split-KV partials).  Calls that run
+/* Bytes of device workspace that tls_sparse_attn_decode(_paged) and
+ * tls_decode_step need for this shape on the current device (the split-KV
+ * partials).  Calls that run
  * concurrently need separate buffers.  The selection stages take a workspace
  * argument too but use none (their keys stay in on-chip memory); they accept
  * NULL.  Returns 0 for an invalid shape (see tls_last_error). */
@@ -212,12 +213,32 @@ TLS_API tls_status tls_select_step(const tls_shape *s, const void *q, const void
                                    int32_t *token_idx_out, float *block_score_out, float *token_score_out,
                                    void *stream);
 
+/* Stages 1-5 in one call: tls_select_step, then tls_sparse_attn_decode on its
+ * token ids, for callers that want the whole decode step.
+ * gist.science (de) section 2.A and (es) section 2.A (the five stages); the
+ * two calls above give the definitions.  Arguments:
+ *   q, meta, slab, label_idx, seq_lens   as in tls_select_step
+ *   K, V                                 as in tls_sparse_attn_decode
+ *   block_idx_out, token_idx_out         device int32 [B][H_kv][k_b] / [k_t] (written)
+ *   out, lse_out                         as in tls_sparse_attn_decode (lse may be NULL)
+ *   block_score_out, token_score_out     as in tls_select_step, or NULL
+ *   ws, ws_bytes                         as in tls_sparse_attn_decode (checked
+ *                                        before anything is enqueued) */
+TLS_API tls_status tls_decode_step(const tls_shape *s, const void *q, const void *meta, const void *slab,
+                                   const int32_t *label_idx, const int32_t *seq_lens, const void *K, const void *V,
+                                   int32_t *block_idx_out, int32_t *token_idx_out, void *out, float *lse_out,
+                                   float *block_score_out, float *token_score_out, void *ws, size_t ws_bytes,
+                                   void *stream);
+
 /* Stage 5: exact attention over the selected tokens.
  * gist.science (es) section 2.A.2: the final attention over the K_t kept tokens
  * at token precision.  For each query head h:
  *   a_t = tau q_h . K[t], o_h = sum_t softmax(a)_t V[t], lse_h = log sum_t exp(a_t)
  * computed by splitting the kept tokens over warps (online softmax, fp32) and
  * merging the partial (max, sum, o) by log-sum-exp.
+ *   ws, ws_bytes  device workspace of tls_workspace_size(s) bytes or more,
+ *              256-byte aligned; calls that run concurrently need separate
+ *              workspaces.
  *   K, V       device [B][H_kv][max_ctx][d_qk] / [..][d_v] (V ignored for MLA)
  *   token_idx  device int32 [B][H_kv][k_t]; entries < 0 or >= max_ctx are skipped
  *   out        device [B][H_q][d_v] in out_dtype

@@ -328,6 +328,41 @@ def full_stage_parity(w: W.Workload, seq_lens=None, out_dtype=0, name=None, inp=
                 step_swaps_t += check_selection(ft[b, g], orc.cand_tok[b, g][oko], orc.cand_scores[b, g][oko], w.k_t,
                                                 what + " tokens")
             check_selection_self_consistent(ft[b, g], cand[ok].astype(np.int32), fts[b, g][ok], what + " tokens")
+    # stages 1-5 in one call (tls_decode_step, the call the benchmark times):
+    # block / token ids and both score arrays identical to the select_step
+    # launch above, attention against the oracle wherever the token ids equal
+    # the oracle's.  Called twice on one workspace, with and without the
+    # optional score outputs.
+    step_groups = 0
+    for call in range(2):
+        db = torch.full((w.batch, w.n_kv_heads, w.k_b), -7, dtype=torch.int32, device="cuda")
+        dt = torch.full((w.batch, w.n_kv_heads, w.k_t), -7, dtype=torch.int32, device="cuda")
+        dbs = torch.zeros((w.batch, w.n_kv_heads, w.n_blocks), dtype=torch.float32, device="cuda")
+        dts = torch.zeros((w.batch, w.n_kv_heads, w.k_b * w.block_size), dtype=torch.float32, device="cuda")
+        odt = torch.int16 if gpu.shape.out_dtype == W.BF16 else torch.float32
+        dout = torch.zeros((w.batch, w.n_q_heads, w.d_v), dtype=odt, device="cuda")
+        dlse = torch.zeros((w.batch, w.n_q_heads), dtype=torch.float32, device="cuda")
+        with_scores = call == 0
+        tls().tls_decode_step(gpu.shape, gpu.q, gpu.meta, gpu.slab, gpu.label, gpu.seq_lens, gpu.K, gpu.V, db, dt,
+                              dout, dlse, dbs if with_scores else None, dts if with_scores else None, gpu.ws)
+        torch.cuda.synchronize()
+        np.testing.assert_array_equal(db.cpu().numpy(), fb, err_msg=f"{name} decode_step block ids, call {call}")
+        np.testing.assert_array_equal(dt.cpu().numpy(), ft, err_msg=f"{name} decode_step token ids, call {call}")
+        if with_scores:
+            np.testing.assert_array_equal(dbs.cpu().numpy().view(np.uint32), fbs.view(np.uint32),
+                                          err_msg=f"{name} decode_step block scores")
+            np.testing.assert_array_equal(dts.cpu().numpy().view(np.uint32), fts.view(np.uint32),
+                                          err_msg=f"{name} decode_step token scores")
+        dout, dlse = gpu.out_f64(dout), dlse.cpu().numpy().astype(np.float64)
+        G = w.group
+        step_groups = 0
+        for b in range(w.batch):
+            for g in range(w.n_kv_heads):
+                if (ft[b, g] == orc.token_idx[b, g]).all():
+                    step_groups += 1
+                    hs = slice(g * G, (g + 1) * G)
+                    check_attention(dout[b, hs], dlse[b, hs], orc.out[b, hs], orc.lse[b, hs],
+                                    f"{name} decode_step attention b{b} g{g} call {call}")
     # chained: the GPU's own selections all the way
     cb, _ = gpu.block_stage(with_scores=False)
     ct, _ = gpu.token_stage(cb, with_scores=False)
@@ -348,7 +383,7 @@ def full_stage_parity(w: W.Workload, seq_lens=None, out_dtype=0, name=None, inp=
                 check_attention(cout[b, hs], clse[b, hs], orc.out[b, hs], orc.lse[b, hs], f"{name} chained b{b} g{g}")
     assert tls().tls_device_error(clear=True) == 0, f"{name}: a kernel's bounded wait gave up"
     res = dict(block_swaps=swaps_b, token_swaps=swaps_t, step_block_swaps=step_swaps_b,
-               step_token_swaps=step_swaps_t, attn_max_abs_err=err,
+               step_token_swaps=step_swaps_t, decode_step_groups_vs_oracle=step_groups, attn_max_abs_err=err,
                chained_groups_identical=same_groups, groups=w.batch * w.n_kv_heads)
     report(name, **res)
     return res

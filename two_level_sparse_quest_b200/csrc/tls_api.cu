@@ -5,6 +5,7 @@
 // and tls_offload.cu.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <chrono>
 #include <mutex>
 #include <cmath>
@@ -158,14 +159,15 @@ struct WsLayout {
   size_t part_off, part_bytes, total;
 };
 
+size_t up256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
 bool ws_layout(const tls_shape *s, bool paged, WsLayout *w) {
-  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
   tls::AttnArgs a = attn_args(s);
   a.paged = paged;
   tls::AttnPlan p;
   if (!tls::attn_plan(a, &p)) return false;
   w->part_off = 0;
-  w->part_bytes = up(p.part_floats * sizeof(float));
+  w->part_bytes = up256(p.part_floats * sizeof(float));
   w->total = w->part_off + w->part_bytes;
   return true;
 }
@@ -463,6 +465,36 @@ tls_status tls_prefetch_diff(const tls_shape *s, int32_t n_slots, const void *ho
   a.n_slots = n_slots;
   a.dtype = s->kv_dtype;
   return cuda_status(tls::launch_prefetch_diff(a, static_cast<cudaStream_t>(stream)), "prefetch_diff launch");
+}
+
+tls_status tls_decode_step(const tls_shape *s, const void *q, const void *meta, const void *slab,
+                           const int32_t *label_idx, const int32_t *seq_lens, const void *K, const void *V,
+                           int32_t *block_idx_out, int32_t *token_idx_out, void *out, float *lse_out,
+                           float *block_score_out, float *token_score_out, void *ws, size_t ws_bytes, void *stream) {
+  tls_status st = check_shape(s);
+  if (st != TLS_OK) return st;
+  if (s->batch == 0) return TLS_OK;
+  CHECK_PTR(q, 16);
+  CHECK_PTR(meta, 16);
+  CHECK_PTR(slab, 16);
+  CHECK_PTR(label_idx, 4);
+  CHECK_PTR(seq_lens, 4);
+  CHECK_PTR(K, 16);
+  if (!s->v_is_k_prefix) CHECK_PTR(V, 16);
+  CHECK_PTR(block_idx_out, 4);
+  CHECK_PTR(token_idx_out, 4);
+  CHECK_PTR(out, 16);
+  if (lse_out && !aligned(lse_out, 4)) return fail(TLS_ERR_INVALID_ARG, "lse_out misaligned");
+  if (block_score_out && !aligned(block_score_out, 4)) return fail(TLS_ERR_INVALID_ARG, "block_score_out misaligned");
+  if (token_score_out && !aligned(token_score_out, 4)) return fail(TLS_ERR_INVALID_ARG, "token_score_out misaligned");
+  const size_t need = tls_workspace_size(s);  // checked before anything is enqueued
+  if (!need) return fail(TLS_ERR_UNSUPPORTED, "no workspace layout for this shape");
+  if (!ws || ws_bytes < need || !aligned(ws, 256))
+    return fail(TLS_ERR_WORKSPACE, "workspace too small or not 256-byte aligned (need %zu bytes)", need);
+  st = tls_select_step(s, q, meta, slab, label_idx, seq_lens, block_idx_out, token_idx_out, block_score_out,
+                       token_score_out, stream);
+  if (st != TLS_OK) return st;
+  return tls_sparse_attn_decode(s, q, K, V, token_idx_out, out, lse_out, ws, ws_bytes, stream);
 }
 
 tls_status tls_wait_event(void *event, int32_t timeout_ms) {
