@@ -246,16 +246,24 @@ def gpu_arm(args, rank, world, local_rank):
         T.tls_decode_step(shape, L.q, L.meta, L.slab, label, seq_lens, L.K, L.V, bidx, tidx, out, lse, None, None,
                           ws, sh)
 
+    bscore = torch.empty((G, w.n_blocks), dtype=torch.float32, device=dev)
+
     def step_stages(L, ev):
-        """The same step as its two calls, with CUDA events around each."""
+        """The same step as its two calls, with CUDA events around each (the
+        selection given a block-score buffer, as tls_decode_step gives it
+        workspace, so that it runs the same launches)."""
         ev[0].record(stream)
-        T.tls_select_step(shape, L.q, L.meta, L.slab, label, seq_lens, bidx, tidx, None, None, sh)
+        T.tls_select_step(shape, L.q, L.meta, L.slab, label, seq_lens, bidx, tidx, bscore, None, sh)
         ev[1].record(stream)
         T.tls_sparse_attn_decode(shape, L.q, L.K, L.V, tidx, out, lse, ws, sh)
         ev[2].record(stream)
 
-    # stages 1-4 (one cluster launch), attention split, log-sum-exp merge
-    launches_per_step = 3
+    # stages 1-4 (one cluster launch; with few groups a block-score launch
+    # first), attention split, log-sum-exp merge
+    groups = w.batch * w.n_kv_heads
+    two_phase = (groups * 8 < 2 * torch.cuda.get_device_properties(dev).multi_processor_count
+                 and algorithmic_bytes(w)["block_summary"] >= 4 << 20 and w.group <= 16)
+    launches_per_step = 3 + (1 if two_phase else 0)
     for i in range(args.warmup):
         step(layers[i % N_LAYERS])
     torch.cuda.synchronize()

@@ -107,7 +107,8 @@ TLS_API const char *tls_last_error(void);
 
 /* Bytes of device workspace that tls_sparse_attn_decode(_paged) and
  * tls_decode_step need for this shape on the current device (the split-KV
- * partials).  Calls that run
+ * partials; tls_decode_step also keeps the step's block scores there before
+ * the attention runs).  Calls that run
  * concurrently need separate buffers.  The selection stages take a workspace
  * argument too but use none (their keys stay in on-chip memory); they accept
  * NULL.  Returns 0 for an invalid shape (see tls_last_error). */
@@ -205,7 +206,12 @@ TLS_API tls_status tls_token_score_topk(const tls_shape *s, const void *q, const
 /* Stages 1-4 in one launch: exactly what tls_block_score_topk followed by
  * tls_token_score_topk compute (same arithmetic, same bits), with each
  * group's thread-block cluster going from its block selection straight to its
- * token stage instead of waiting for every group's block selection.
+ * token stage instead of waiting for every group's block selection.  With
+ * few groups (fewer than two clusters per SM), at least 4 MB of block
+ * summary, at most 16 query heads per KV head and block_score_out given, the
+ * block scores are first computed by a grid over all SMs into block_score_out
+ * and the clusters select from them (two launches, same bits): one cluster
+ * per group alone cannot keep HBM busy.
  * Arguments as in those two calls; block_idx_out is written and then read
  * back by the same launch.  block_score_out / token_score_out may be NULL. */
 TLS_API tls_status tls_select_step(const tls_shape *s, const void *q, const void *meta, const void *slab,

@@ -221,9 +221,12 @@ size_t tls_workspace_size(const tls_shape *s) {
     fail(TLS_ERR_UNSUPPORTED, "no attention plan for this shape");
     return 0;
   }
+  size_t total = w.total;
   WsLayout wp;
-  if (!s->v_is_k_prefix && ws_layout(s, true, &wp) && wp.total > w.total) return wp.total;
-  return w.total;
+  if (!s->v_is_k_prefix && ws_layout(s, true, &wp) && wp.total > total) total = wp.total;
+  // tls_decode_step keeps the step's block scores here before the attention runs
+  const size_t scores = up256(static_cast<size_t>(s->batch) * s->n_kv_heads * n_blocks_max(s) * sizeof(float));
+  return std::max(total, scores);
 }
 
 size_t tls_slab_bytes(const tls_shape *s) {
@@ -321,9 +324,24 @@ tls_status tls_token_score_topk(const tls_shape *s, const void *q, const void *s
   return cuda_status(tls::launch_token_select(a, static_cast<cudaStream_t>(stream)), "token_select launch");
 }
 
+// Stages 1-4.  scratch: room for the step's block scores when the caller
+// passes no block_score_out (tls_decode_step lends its workspace), or NULL.
+static tls_status select_step_impl(const tls_shape *s, const void *q, const void *meta, const void *slab,
+                                   const int32_t *label_idx, const int32_t *seq_lens, int32_t *block_idx_out,
+                                   int32_t *token_idx_out, float *block_score_out, float *token_score_out,
+                                   float *scratch, void *stream);
+
 tls_status tls_select_step(const tls_shape *s, const void *q, const void *meta, const void *slab,
                            const int32_t *label_idx, const int32_t *seq_lens, int32_t *block_idx_out,
                            int32_t *token_idx_out, float *block_score_out, float *token_score_out, void *stream) {
+  return select_step_impl(s, q, meta, slab, label_idx, seq_lens, block_idx_out, token_idx_out, block_score_out,
+                          token_score_out, nullptr, stream);
+}
+
+static tls_status select_step_impl(const tls_shape *s, const void *q, const void *meta, const void *slab,
+                                   const int32_t *label_idx, const int32_t *seq_lens, int32_t *block_idx_out,
+                                   int32_t *token_idx_out, float *block_score_out, float *token_score_out,
+                                   float *scratch, void *stream) {
   tls_status st = check_shape(s);
   if (st != TLS_OK) return st;
   if (s->batch == 0) return TLS_OK;
@@ -347,6 +365,18 @@ tls_status tls_select_step(const tls_shape *s, const void *q, const void *meta, 
     st = cuda_status(tls::launch_block_select(a, cs), "block_select launch");
     if (st != TLS_OK) return st;
     return cuda_status(tls::launch_token_select(t, cs), "token_select launch");
+  }
+  // Few groups: too few clusters to keep HBM busy streaming the summary, so a
+  // grid over all SMs scores every block first and the clusters only select.
+  float *scores = block_score_out ? block_score_out : scratch;
+  const size_t summary_bytes = static_cast<size_t>(s->batch) * s->n_kv_heads * n_blocks_max(s) * 2 * s->d_qk *
+                               (s->kv_dtype == TLS_BF16 ? 2 : 4);
+  if (scores && tls::select_two_phase(s->batch * s->n_kv_heads, s->n_q_heads / s->n_kv_heads, device_sms(),
+                                      summary_bytes)) {
+    a.scores = scores;
+    st = cuda_status(tls::launch_block_scores(a, device_sms(), cs), "block_scores launch");
+    if (st != TLS_OK) return st;
+    a.from_scores = 1;
   }
   return cuda_status(tls::launch_select_step(a, t, cs), "select_step launch");
 }
@@ -491,8 +521,10 @@ tls_status tls_decode_step(const tls_shape *s, const void *q, const void *meta, 
   if (!need) return fail(TLS_ERR_UNSUPPORTED, "no workspace layout for this shape");
   if (!ws || ws_bytes < need || !aligned(ws, 256))
     return fail(TLS_ERR_WORKSPACE, "workspace too small or not 256-byte aligned (need %zu bytes)", need);
-  st = tls_select_step(s, q, meta, slab, label_idx, seq_lens, block_idx_out, token_idx_out, block_score_out,
-                       token_score_out, stream);
+  // the block scores may borrow the workspace: they are consumed by the
+  // selection launch before the attention writes its partials there
+  st = select_step_impl(s, q, meta, slab, label_idx, seq_lens, block_idx_out, token_idx_out, block_score_out,
+                        token_score_out, static_cast<float *>(ws), stream);
   if (st != TLS_OK) return st;
   return tls_sparse_attn_decode(s, q, K, V, token_idx_out, out, lse_out, ws, ws_bytes, stream);
 }

@@ -85,9 +85,16 @@ struct BlockScoreArgs {
   int batch, n_q_heads, n_kv_heads, d, block_size, n_blocks_max, max_ctx, k_b, dtype;
   int *err;           // the library's device error word
   int agg;            // 0: sum of the heads' bounds, 1: their max
+  int from_scores;    // 1: scores already hold the step's block scores (the cluster only selects)
 };
 // Block score and top-K_b in one launch (one thread-block cluster per group).
 cudaError_t launch_block_select(const BlockScoreArgs &a, cudaStream_t st);
+// Whether the two-phase selection pays off for this many groups on this
+// device: the block summary is then streamed by a grid over all SMs into
+// a.scores first, and the clusters select from those scores.
+bool select_two_phase(int groups, int heads_per_group, int num_sms, size_t summary_bytes);
+// Phase 1 of the two-phase selection: every group's block scores into a.scores.
+cudaError_t launch_block_scores(const BlockScoreArgs &a, int num_sms, cudaStream_t st);
 
 struct TokenArgs {
   const void *q;

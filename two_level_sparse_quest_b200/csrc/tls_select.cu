@@ -45,7 +45,7 @@ constexpr int kThreads = 256;
 // byte).  NCH: 16-byte chunks per summary row (2 * d * bytes / 16).  The first
 // rows' loads are issued before the head fold so that the query reads
 // overlap them.
-template <typename E, int NCH>
+template <typename E, int NCH, bool KEYS = true>
 __device__ __forceinline__ void score_blocks(const BlockScoreArgs &a, int group, int nb, int r0, int r1, float *qpm,
                                              uint32_t *keys, int *hist) {
   constexpr int EPC = E::kEPC;
@@ -115,9 +115,11 @@ __device__ __forceinline__ void score_blocks(const BlockScoreArgs &a, int group,
       const int row = rb + u * STEP + sub;
       if (cl == 0 && row < r1) {
         const bool valid = row < nb;
-        const uint32_t key = valid ? max(score_key(acc), 1u) : 0u;
-        keys[row - r0] = key;
-        hist_add(hist, key, valid);
+        if constexpr (KEYS) {
+          const uint32_t key = valid ? max(score_key(acc), 1u) : 0u;
+          keys[row - r0] = key;
+          hist_add(hist, key, valid);
+        }
         if (out) out[row] = valid ? acc : -INFINITY;
       }
     }
@@ -127,6 +129,42 @@ __device__ __forceinline__ void score_blocks(const BlockScoreArgs &a, int group,
 #pragma unroll
         for (int j = 0; j < CPL; ++j) v[u][j] = nv[u][j];
     }
+  }
+}
+
+// The stage-1 keys of rows [r0, r1) from block scores a previous launch
+// wrote (the two-phase selection): the same keys score_blocks makes.
+__device__ __forceinline__ void keys_from_scores(const BlockScoreArgs &a, int group, int nb, int r0, int r1,
+                                                 uint32_t *keys, int *hist) {
+  const float *sc = a.scores + static_cast<size_t>(group) * a.n_blocks_max;
+  for (int row = r0 + threadIdx.x; row < r1; row += kThreads) {
+    const bool valid = row < nb;
+    const uint32_t key = valid ? max(score_key(__ldcg(sc + row)), 1u) : 0u;
+    keys[row - r0] = key;
+    hist_add(hist, key, valid);
+  }
+}
+
+// Phase 1 of the two-phase selection: CTA c scores the c-th equal range of
+// all groups' summary rows (a range may cross into the next group; the
+// query fold is redone per group) into a.scores, with score_blocks' arithmetic.
+template <typename E, int NCH>
+__global__ void __launch_bounds__(kThreads, NCH > 32 ? 2 : 4) block_scores_kernel(BlockScoreArgs a, int rows_per_cta) {
+  extern __shared__ float qpm[];  // [2d]
+  grid_dependency_wait();
+  const long long total = static_cast<long long>(a.batch) * a.n_kv_heads * a.n_blocks_max;
+  long long r0 = static_cast<long long>(blockIdx.x) * rows_per_cta;
+  const long long r1 = std::min(r0 + rows_per_cta, total);
+  while (r0 < r1) {
+    const int group = static_cast<int>(r0 / a.n_blocks_max);
+    const long long gbase = static_cast<long long>(group) * a.n_blocks_max;
+    const long long gend = std::min(r1, gbase + a.n_blocks_max);
+    const int sq = min(max(a.seq_lens[group / a.n_kv_heads], 0), a.max_ctx);
+    const int nb = (sq + a.block_size - 1) / a.block_size;
+    score_blocks<E, NCH, false>(a, group, nb, static_cast<int>(r0 - gbase), static_cast<int>(gend - gbase), qpm,
+                                nullptr, nullptr);
+    __syncthreads();  // qpm is folded again for the next group
+    r0 = gend;
   }
 }
 
@@ -382,7 +420,8 @@ __global__ void __launch_bounds__(kThreads, NCH > 32 ? 2 : token_min_blocks<RCH,
   // ---- stages 1 + 2
   const int r0 = rank * rows_per_cta;
   const int r1 = min(r0 + rows_per_cta, a.n_blocks_max);
-  score_blocks<E, NCH>(a, group, nb, r0, r1, qpm, bkeys, SB.hist);
+  if (a.from_scores) keys_from_scores(a, group, nb, r0, r1, bkeys, SB.hist);
+  else score_blocks<E, NCH>(a, group, nb, r0, r1, qpm, bkeys, SB.hist);
   int32_t *bout = a.block_idx + static_cast<size_t>(group) * a.k_b;
   cluster_topk<kThreads, CS, kSliceCap>(
       bkeys, max(r1 - r0, 0), a.k_b, bout, a.k_b, [r0](int i) { return r0 + i; }, SB, a.err);
@@ -529,6 +568,46 @@ cudaError_t launch_token_select(const TokenArgs &a, cudaStream_t st) {
     case 2: return a.dtype == 1 ? run_token_select<BF16, BF16, 2>(a, st) : run_token_select<F32, F32, 2>(a, st);
     case 4: return a.dtype == 1 ? run_token_select<BF16, BF16, 4>(a, st) : run_token_select<F32, F32, 4>(a, st);
     case 8: return a.dtype == 1 ? run_token_select<BF16, BF16, 8>(a, st) : run_token_select<F32, F32, 8>(a, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+bool select_two_phase(int groups, int heads_per_group, int num_sms, size_t summary_bytes) {
+  // One cluster of kClusterSize CTAs per group: with fewer clusters than fill
+  // the SMs twice over, the summary stream is short of loads in flight.  Below
+  // a few MB of summary the extra launch costs more than it saves, and with
+  // many heads per group every phase-1 CTA pays the query fold over all of
+  // them (measured: gqa48k 21.9 -> 18.4 us; the 64-head latent 33.8 -> 37.7 us).
+  return static_cast<long long>(groups) * kClusterSize < 2LL * num_sms && summary_bytes >= (size_t(4) << 20) &&
+         heads_per_group <= 16;
+}
+
+namespace {
+template <typename E, int NCH>
+cudaError_t run_block_scores(const BlockScoreArgs &a, int num_sms, cudaStream_t st) {
+  const long long total = static_cast<long long>(a.batch) * a.n_kv_heads * a.n_blocks_max;
+  const int ctas = static_cast<int>(std::max<long long>(1, std::min<long long>(4LL * num_sms, total)));
+  const int rows = static_cast<int>((total + ctas - 1) / ctas);
+  const int grid = static_cast<int>((total + rows - 1) / rows);
+  const size_t smem = 2 * static_cast<size_t>(a.d) * sizeof(float);
+  return launch_pdl(block_scores_kernel<E, NCH>, dim3(grid), dim3(kThreads), smem, st, a, rows);
+}
+}  // namespace
+
+cudaError_t launch_block_scores(const BlockScoreArgs &a, int num_sms, cudaStream_t st) {
+  if (!a.scores) return cudaErrorInvalidValue;
+  const int nch = 2 * a.d * (a.dtype == 1 ? 2 : 4) / 16;
+  if (a.dtype == 1) {
+    switch (nch) {
+      case 16: return run_block_scores<BF16, 16>(a, num_sms, st);
+      case 32: return run_block_scores<BF16, 32>(a, num_sms, st);
+      case 144: return run_block_scores<BF16, 144>(a, num_sms, st);
+    }
+  } else {
+    switch (nch) {
+      case 32: return run_block_scores<F32, 32>(a, num_sms, st);
+      case 64: return run_block_scores<F32, 64>(a, num_sms, st);
+    }
   }
   return cudaErrorInvalidValue;
 }
