@@ -123,9 +123,17 @@ def test_block_aggregation_field_is_checked(T):
     s = good_shape(T)
     s.block_agg = 2
     assert call_block(T, s) == T.TLS_ERR_INVALID_ARG and "block_agg" in T.tls_last_error()
+    # the latent shape takes the max-over-heads scores on the tensor cores, which need room for
+    # the scores: without block_score_out or a workspace the call is refused before any launch
     mla = good_shape(T, v_is_k_prefix=True, n_q_heads=64, n_kv_heads=1, d_qk=576, d_v=512, n_label=32)
     mla.block_agg = 1
-    assert call_block(T, mla) == T.TLS_ERR_UNSUPPORTED
+    assert call_block(T, mla, ws=(None, 0)) == T.TLS_ERR_WORKSPACE and "block_score_out" in T.tls_last_error()
+    big = good_shape(T, v_is_k_prefix=True, n_q_heads=128, n_kv_heads=1, d_qk=576, d_v=512, n_label=32)
+    big.block_agg = 1
+    assert call_block(T, big) == T.TLS_ERR_UNSUPPORTED
+    f32 = good_shape(T, kv_dtype=T.TLS_F32, n_q_heads=16, n_kv_heads=1, d_qk=64, d_v=64)
+    f32.block_agg = 1
+    assert call_block(T, f32) == T.TLS_ERR_UNSUPPORTED
 
 
 def test_group_sizes(T):
@@ -134,9 +142,10 @@ def test_group_sizes(T):
         assert T.tls_workspace_size(good_shape(T, n_q_heads=G, n_kv_heads=1, d_qk=64, d_v=64)) > 0
     st = call_block(T, good_shape(T, n_q_heads=24, n_kv_heads=1))
     assert st == T.TLS_ERR_UNSUPPORTED and "group size" in T.tls_last_error()
+    # max-over-heads with 16 heads per group: the tensor-core path, which needs room for the scores
     mq = good_shape(T, n_q_heads=16, n_kv_heads=1)
     mq.block_agg = 1
-    assert call_block(T, mq) == T.TLS_ERR_UNSUPPORTED and "up to 8 heads" in T.tls_last_error()
+    assert call_block(T, mq, ws=(None, 0)) == T.TLS_ERR_WORKSPACE and "16 heads" in T.tls_last_error()
 
 
 def test_int8_slab_field_and_size(T):

@@ -113,6 +113,17 @@ AGG_MAX = {
     "agg_max_f32_ragged": (W.WORKLOADS["tiny_gqa4k_f32"].with_(batch=3, ctx=1000, k_b=8, k_t=100, n_q_heads=8,
                                                                 block_agg=1), [1000, 777, 33]),
     "agg_max_full_gqa96k_b8": (W.WORKLOADS["gqa96k_b8_bf16"].with_(block_agg=1), None),
+    # more heads per group than the CUDA-core variant takes: the per-head bounds as a tcgen05 GEMM
+    "agg_max_bf16_g16": (W.WORKLOADS["gqa48k_bf16"].with_(batch=2, n_q_heads=32, n_kv_heads=2, ctx=4096, k_b=24,
+                                                          k_t=300, block_agg=1), [4096, 2900]),
+    "agg_max_bf16_mqa_g32": (W.WORKLOADS["gqa48k_bf16"].with_(batch=2, n_q_heads=32, n_kv_heads=1, ctx=4096, k_b=24,
+                                                              k_t=300, block_agg=1), [4096, 1777]),
+    "agg_max_bf16_mqa_g64_d64": (W.WORKLOADS["gqa48k_bf16"].with_(batch=3, n_q_heads=64, n_kv_heads=1, d_qk=64,
+                                                                  d_v=64, ctx=3000, k_b=20, k_t=211, block_agg=1),
+                                 [3000, 17, 2500]),
+    "agg_max_mla_small": (W.WORKLOADS["mla64k_b4_bf16"].with_(batch=2, ctx=4096, k_b=16, k_t=300, n_needles=4,
+                                                              block_agg=1), [4096, 3000]),
+    "agg_max_full_mla64k_b4": (W.WORKLOADS["mla64k_b4_bf16"].with_(block_agg=1), None),
 }
 
 

@@ -76,8 +76,8 @@ tls_status check_shape(const tls_shape *s) {
   if (s->d_qk < 1 || s->d_v < 1) return fail(TLS_ERR_INVALID_ARG, "d_qk and d_v must be >= 1");
   if (s->v_is_k_prefix && s->d_v > s->d_qk) return fail(TLS_ERR_INVALID_ARG, "v_is_k_prefix needs d_v <= d_qk");
   if (s->block_agg != 0 && s->block_agg != 1) return fail(TLS_ERR_INVALID_ARG, "block_agg %d", s->block_agg);
-  if (s->block_agg == 1 && s->v_is_k_prefix)
-    return fail(TLS_ERR_UNSUPPORTED, "max-over-heads block aggregation supports GQA shapes only");
+  if (s->block_agg == 1 && s->v_is_k_prefix && s->n_q_heads / s->n_kv_heads > 64)
+    return fail(TLS_ERR_UNSUPPORTED, "max-over-heads block aggregation supports up to 64 heads per latent");
   if (static_cast<long long>(s->batch) * s->n_kv_heads > 65535)
     return fail(TLS_ERR_UNSUPPORTED, "batch * n_kv_heads > 65535");
   const int G = s->n_q_heads / s->n_kv_heads;
@@ -89,8 +89,8 @@ tls_status check_shape(const tls_shape *s) {
       return fail(TLS_ERR_UNSUPPORTED, "GQA supports d_qk = d_v in {64, 128} (got %d, %d)", s->d_qk, s->d_v);
     if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16 && G != 32 && G != 64)
       return fail(TLS_ERR_UNSUPPORTED, "GQA group size %d not in {1,2,4,8,16,32,64}", G);
-    if (s->block_agg == 1 && G > 8)
-      return fail(TLS_ERR_UNSUPPORTED, "max-over-heads block aggregation supports groups of up to 8 heads");
+    if (s->block_agg == 1 && G > 8 && s->kv_dtype != TLS_BF16)
+      return fail(TLS_ERR_UNSUPPORTED, "max-over-heads block aggregation of fp32 keys supports up to 8 heads per group");
   }
   if (n_blocks_max(s) > tls::kMaxSelectKeys)
     return fail(TLS_ERR_UNSUPPORTED, "ceil(max_ctx / block_size) = %d > %d", n_blocks_max(s), tls::kMaxSelectKeys);
@@ -284,6 +284,27 @@ tls_status tls_append_tokens(const tls_shape *s, const void *K, const int32_t *o
   return cuda_status(tls::launch_append_tokens(a, static_cast<cudaStream_t>(stream)), "append_tokens launch");
 }
 
+// block_agg 1: the per-head bounds as a tcgen05 GEMM into `scores` (then the
+// clusters only select, a.from_scores), when the shape allows it and there is
+// room for the scores; otherwise the CUDA-core path (up to 8 heads per group).
+// Returns TLS_OK with a.from_scores set when the scores were launched.
+static tls_status agg_max_scores(const tls_shape *s, tls::BlockScoreArgs &a, float *scores, cudaStream_t cs) {
+  const int G = s->n_q_heads / s->n_kv_heads;
+  if (scores && tls::block_scores_max_tc_supported(s->kv_dtype, s->d_qk, G)) {
+    a.scores = scores;
+    tls_status st = cuda_status(tls::launch_block_scores_max_tc(a, device_sms(), cs), "block_scores_max_tc launch");
+    if (st != TLS_OK) return st;
+    a.from_scores = 1;
+    return TLS_OK;
+  }
+  if (G > 8 || s->v_is_k_prefix)
+    return fail(TLS_ERR_WORKSPACE,
+                "max-over-heads block scores with %d heads per group need block_score_out or a workspace of "
+                "tls_workspace_size bytes",
+                G);
+  return TLS_OK;  // CUDA-core path
+}
+
 tls_status tls_block_score_topk(const tls_shape *s, const void *q, const void *meta, const int32_t *seq_lens,
                                 int32_t *block_idx_out, float *block_score_out, void *ws, size_t ws_bytes,
                                 void *stream) {
@@ -295,12 +316,19 @@ tls_status tls_block_score_topk(const tls_shape *s, const void *q, const void *m
   CHECK_PTR(seq_lens, 4);
   CHECK_PTR(block_idx_out, 4);
   if (block_score_out && !aligned(block_score_out, 4)) return fail(TLS_ERR_INVALID_ARG, "block_score_out misaligned");
-  (void)ws;  // the selection keeps its keys in on-chip memory: no workspace
-  (void)ws_bytes;
   tls::BlockScoreArgs a{q, meta, seq_lens, block_score_out, block_idx_out, s->batch, s->n_q_heads, s->n_kv_heads,
                         s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->k_b, s->kv_dtype,
                         tls::device_error_word(), s->block_agg};
-  return cuda_status(tls::launch_block_select(a, static_cast<cudaStream_t>(stream)), "block_select launch");
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  if (s->block_agg == 1) {
+    // the scores of the tensor-core path go to block_score_out, else to the workspace
+    const size_t need = static_cast<size_t>(s->batch) * s->n_kv_heads * n_blocks_max(s) * sizeof(float);
+    float *scores = block_score_out ? block_score_out
+                                    : (ws && ws_bytes >= need && aligned(ws, 16) ? static_cast<float *>(ws) : nullptr);
+    st = agg_max_scores(s, a, scores, cs);
+    if (st != TLS_OK) return st;
+  }
+  return cuda_status(tls::launch_block_select(a, cs), "block_select launch");
 }
 
 tls_status tls_token_score_topk(const tls_shape *s, const void *q, const void *slab, const int32_t *label_idx,
@@ -361,7 +389,12 @@ static tls_status select_step_impl(const tls_shape *s, const void *q, const void
                    s->n_kv_heads, s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->n_label, s->k_b, s->k_t,
                    s->kv_dtype, err, slab_scales(s, slab)};
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  if (s->block_agg == 1) {  // the max-over-heads variant runs as the two separate launches
+  if (s->block_agg == 1) {
+    st = agg_max_scores(s, a, block_score_out ? block_score_out : scratch, cs);
+    if (st != TLS_OK) return st;
+    if (a.from_scores)  // tensor-core scores: the cluster launch selects blocks, then tokens
+      return cuda_status(tls::launch_select_step(a, t, cs), "select_step launch");
+    // CUDA-core max-over-heads scores: the two separate launches
     st = cuda_status(tls::launch_block_select(a, cs), "block_select launch");
     if (st != TLS_OK) return st;
     return cuda_status(tls::launch_token_select(t, cs), "token_select launch");

@@ -95,6 +95,11 @@ cudaError_t launch_block_select(const BlockScoreArgs &a, cudaStream_t st);
 bool select_two_phase(int groups, int heads_per_group, int num_sms, size_t summary_bytes);
 // Phase 1 of the two-phase selection: every group's block scores into a.scores.
 cudaError_t launch_block_scores(const BlockScoreArgs &a, int num_sms, cudaStream_t st);
+// The max-over-heads block scores (block_agg 1) of every group into a.scores,
+// as a tcgen05 GEMM [blocks x 2d] . [2d x heads] with a row maximum (bf16,
+// d in {64, 128, 576}, up to 64 heads per group).
+bool block_scores_max_tc_supported(int dtype, int d, int heads_per_group);
+cudaError_t launch_block_scores_max_tc(const BlockScoreArgs &a, int num_sms, cudaStream_t st);
 
 struct TokenArgs {
   const void *q;

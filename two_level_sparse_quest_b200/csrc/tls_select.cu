@@ -348,7 +348,8 @@ __global__ void __launch_bounds__(kThreads, NCH > 32 ? 2 : 4) block_select_kerne
   const int nb = (sq + a.block_size - 1) / a.block_size;
   const int r0 = rank * rows_per_cta;
   const int r1 = min(r0 + rows_per_cta, a.n_blocks_max);
-  if constexpr (AGG_MAX) score_blocks_max<E, NCH>(a, group, nb, r0, r1, qpm, keys, S.hist);
+  if (a.from_scores) keys_from_scores(a, group, nb, r0, r1, keys, S.hist);
+  else if constexpr (AGG_MAX) score_blocks_max<E, NCH>(a, group, nb, r0, r1, qpm, keys, S.hist);
   else score_blocks<E, NCH>(a, group, nb, r0, r1, qpm, keys, S.hist);
   cluster_topk<kThreads, CS, kSliceCap>(
       keys, max(r1 - r0, 0), a.k_b, a.block_idx + static_cast<size_t>(group) * a.k_b, a.k_b,
@@ -477,6 +478,7 @@ cudaError_t run_block_select_agg(const BlockScoreArgs &a, cudaStream_t st) {
 }
 template <typename E, int NCH>
 cudaError_t run_block_select(const BlockScoreArgs &a, cudaStream_t st) {
+  if (a.from_scores) return run_block_select_agg<E, NCH, false>(a, st);  // selection only: no query in smem
   if (a.agg == 1) {
     if constexpr (NCH <= 64) return run_block_select_agg<E, NCH, true>(a, st);
     return cudaErrorInvalidValue;  // latent shapes: max aggregation not offered
