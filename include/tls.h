@@ -83,15 +83,17 @@ typedef struct tls_shape {
   int32_t out_dtype;     /* tls_dtype of the attention output                            */
   float softmax_scale;   /* tau; <= 0 selects 1/sqrt(d_qk)                               */
   int32_t block_agg;     /* block score over the group's heads: 0 = sum of the heads'
-                          * bounds (the method), 1 = their maximum (a variant; GQA only)  */
+                          * bounds (the method), 1 = their maximum (a variant)           */
   int32_t slab_bits;     /* label slab: 0 = the K dtype; 8 = int8 codes with one fp32 scale
                           * per (sequence, KV head, label channel) (bf16 K, r in {16,32,64}) */
 } tls_shape;
 
 /* Supported shapes (others return TLS_ERR_UNSUPPORTED):
  *   GQA/MQA/MHA: v_is_k_prefix = 0, kv_dtype F32 or BF16, d_qk = d_v in {64, 128},
- *                G = n_q_heads / n_kv_heads in {1, 2, 4, 8, 16, 32, 64} (block_agg 1:
- *                G <= 8);
+ *                G = n_q_heads / n_kv_heads in {1, 2, 4, 8, 16, 32, 64};
+ *   block_agg 1: bf16 with G <= 64 (GQA, or the latent shape), the per-head
+ *                bounds as a tensor-core GEMM whose scores need room (see
+ *                tls_block_score_topk); fp32 with G <= 8 on CUDA cores;
  *   MLA:         v_is_k_prefix = 1, kv_dtype BF16, d_qk = 576, d_v = 512,
  *                G a multiple of 4 up to 128;
  *   block_size >= 1, ceil(max_ctx / bs) <= 16384 blocks, 1 <= k_b <= 1024,
@@ -175,9 +177,15 @@ TLS_API tls_status tls_append_tokens(const tls_shape *s, const void *K, const in
  *   block_idx_out  device int32 [B][H_kv][k_b], ascending block ids, -1 padded
  *   block_score_out device fp32 [B][H_kv][ceil(max_ctx/bs)] or NULL; blocks at or
  *                  beyond ceil(seq_len/bs) hold -inf
- *   ws, ws_bytes   unused (may be NULL / 0)
+ *   ws, ws_bytes   unused (may be NULL / 0), except for block_agg 1 with bf16
+ *                  keys: the per-head bounds then run as a tcgen05 GEMM whose
+ *                  block scores go to block_score_out, or when that is NULL to
+ *                  ws (at least B*H_kv*ceil(max_ctx/bs)*4 bytes, 16-byte
+ *                  aligned); with neither, groups of up to 8 heads take the
+ *                  CUDA-core path and larger ones return TLS_ERR_WORKSPACE.
  * One launch: the blocks of each group are scored by one thread-block cluster
- * whose CTAs then select the top K_b together. */
+ * whose CTAs then select the top K_b together (block_agg 1 on the tensor
+ * cores: the score launch, then the cluster launch selecting from the scores). */
 TLS_API tls_status tls_block_score_topk(const tls_shape *s, const void *q, const void *meta, const int32_t *seq_lens,
                                 int32_t *block_idx_out, float *block_score_out, void *ws, size_t ws_bytes,
                                 void *stream);
@@ -213,7 +221,9 @@ TLS_API tls_status tls_token_score_topk(const tls_shape *s, const void *q, const
  * and the clusters select from them (two launches, same bits): one cluster
  * per group alone cannot keep HBM busy.
  * Arguments as in those two calls; block_idx_out is written and then read
- * back by the same launch.  block_score_out / token_score_out may be NULL. */
+ * back by the same launch.  block_score_out / token_score_out may be NULL.
+ * block_agg 1 with bf16 keys and more than 8 heads per group (or the latent
+ * shape) needs block_score_out (tls_decode_step lends its workspace). */
 TLS_API tls_status tls_select_step(const tls_shape *s, const void *q, const void *meta, const void *slab,
                                    const int32_t *label_idx, const int32_t *seq_lens, int32_t *block_idx_out,
                                    int32_t *token_idx_out, float *block_score_out, float *token_score_out,
