@@ -215,7 +215,7 @@ def gpu_arm(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    base = W.WORKLOADS[args.workload].with_(slab_bits=args.slab_bits)
+    base = W.WORKLOADS[args.workload].with_(slab_bits=args.slab_bits, block_agg=args.block_agg)
     w = rank_workload(base, rank)
     shape = T.shape_from_workload(w)
     inp = W.make_decode_inputs(w)
@@ -263,7 +263,8 @@ def gpu_arm(args, rank, world, local_rank):
     groups = w.batch * w.n_kv_heads
     two_phase = (groups * 8 < 2 * torch.cuda.get_device_properties(dev).multi_processor_count
                  and algorithmic_bytes(w)["block_summary"] >= 4 << 20 and w.group <= 16)
-    launches_per_step = 3 + (1 if two_phase else 0)
+    # max-over-heads: a score launch (or the two separate selection launches) before the rest
+    launches_per_step = 3 + (1 if (two_phase or w.block_agg == 1) else 0)
     for i in range(args.warmup):
         step(layers[i % N_LAYERS])
     torch.cuda.synchronize()
@@ -395,6 +396,7 @@ def gpu_arm(args, rank, world, local_rank):
             "workload": args.workload, "batch": w.batch, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
             "d_qk": w.d_qk, "d_v": w.d_v, "ctx": w.ctx, "block_size": w.block_size, "k_b": w.k_b, "k_t": w.k_t,
             "n_label": w.n_label, "out_dtype": "f32", "label_slab": "int8" if w.slab_bits == 8 else "kv dtype",
+            "block_agg": "max over heads" if w.block_agg == 1 else "sum over heads",
             "l2": f"inputs larger than L2: {N_LAYERS} layer copies rotated, {N_LAYERS * ab['total'] / 1e6:.0f} MB "
                   f"of algorithmic bytes per rotation (L2 126 MB)",
             "algorithmic_bytes_per_step": ab["total"],
@@ -717,6 +719,8 @@ def main():
                     help="time full-attention decode (all tokens selected) of the workload, for context")
     ap.add_argument("--offload", action="store_true",
                     help="time the offload engine on the streaming workload instead (one JSON line of its own)")
+    ap.add_argument("--block-agg", type=int, default=0, choices=[0, 1],
+                    help="block score over a group's heads: 0 = the sum (the method), 1 = the maximum (variant)")
     ap.add_argument("--slab-bits", type=int, default=0, choices=[0, 8],
                     help="label slab storage: 0 = the K dtype (the method), 8 = int8 codes + per-channel scales")
     ap.add_argument("--layers", type=int, default=0,
