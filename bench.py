@@ -78,10 +78,18 @@ def read_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "source": "fallback"}
 
 
-def kernel_source_hash() -> str:
+# the sources each stage's kernels are built from (a profile of a stage stays
+# valid while these are unchanged)
+STAGE_SOURCES = {
+    "stage_select": ["tls_select.cu", "tls_device.cuh", "tls_internal.h"],
+    "stage_attn": ["tls_attn.cu", "tls_attn_mma.cu", "tls_mma.cuh", "tls_device.cuh", "tls_internal.h"],
+}
+
+
+def kernel_source_hash(files=None) -> str:
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "two_level_sparse_quest_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(files if files is not None else os.listdir(csrc)):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -89,14 +97,14 @@ def kernel_source_hash() -> str:
 
 def read_profile(stage: str):
     """The committed ncu summary entry of a stage (profiles/traffic.json), only
-    if it was taken on the kernel sources as they are now."""
+    if it was taken on the stage's kernel sources as they are now."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         d = json.load(f)
     ent = d.get(stage)
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(STAGE_SOURCES.get(stage)):
         return None
     return ent
 

@@ -36,7 +36,7 @@ def test_traffic_is_only_reported_for_the_current_kernel_sources(tmp_path, monke
     prof = tmp_path / "profiles"
     prof.mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
-    monkeypatch.setattr(bench, "kernel_source_hash", lambda: "abc")
+    monkeypatch.setattr(bench, "kernel_source_hash", lambda files=None: "abc")
     (prof / "traffic.json").write_text(json.dumps({"stage_select": {"bytes_per_launch": 5.0, "source_hash": "abc"}}))
     assert bench.read_traffic("stage_select") == 5.0
     assert bench.read_traffic("stage_attn") is None
