@@ -273,6 +273,13 @@ def gpu_arm(args, rank, world, local_rank):
                  and algorithmic_bytes(w)["block_summary"] >= 4 << 20 and w.group <= 16)
     # max-over-heads: a score launch (or the two separate selection launches) before the rest
     launches_per_step = 3 + (1 if (two_phase or w.block_agg == 1) else 0)
+    # The clock sampler starts (and settles) before the warm-up, so that the
+    # GPU does not sit idle between the warm-up and the timed region and the
+    # timed steps start at the clocks the warm-up brought it to.
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+    sampler = ClockSampler(int(vis[local_rank]) if local_rank < len(vis) and vis[local_rank].isdigit() else local_rank)
+    if rank == 0:
+        sampler.start()
     for i in range(args.warmup):
         step(layers[i % N_LAYERS])
     torch.cuda.synchronize()
@@ -281,10 +288,6 @@ def gpu_arm(args, rank, world, local_rank):
     # within and across steps are chained by programmatic dependent launch.
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
-    sampler = ClockSampler(int(vis[local_rank]) if local_rank < len(vis) and vis[local_rank].isdigit() else local_rank)
-    if rank == 0:
-        sampler.start()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()

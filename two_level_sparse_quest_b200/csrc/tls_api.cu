@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <chrono>
 #include <mutex>
 #include <cmath>
@@ -172,6 +173,17 @@ bool ws_layout(const tls_shape *s, bool paged, WsLayout *w) {
   return true;
 }
 
+// tls_decode_step's workspace: the attention partials (or, before the
+// attention runs, the step's block scores) from offset 0, then one readiness
+// word per group at this offset.
+size_t ready_words_offset(const tls_shape *s) {
+  WsLayout w, wp;
+  size_t body = ws_layout(s, false, &w) ? w.total : 0;
+  if (!s->v_is_k_prefix && ws_layout(s, true, &wp)) body = std::max(body, wp.total);
+  const size_t scores = up256(static_cast<size_t>(s->batch) * s->n_kv_heads * n_blocks_max(s) * sizeof(float));
+  return up256(std::max(body, scores));
+}
+
 // The library's device error word: one int per GPU, zero until a kernel's
 // bounded wait gives up (bits kErrAttnWait, kErrSelectWait).
 __device__ int g_device_error;
@@ -221,12 +233,7 @@ size_t tls_workspace_size(const tls_shape *s) {
     fail(TLS_ERR_UNSUPPORTED, "no attention plan for this shape");
     return 0;
   }
-  size_t total = w.total;
-  WsLayout wp;
-  if (!s->v_is_k_prefix && ws_layout(s, true, &wp) && wp.total > total) total = wp.total;
-  // tls_decode_step keeps the step's block scores here before the attention runs
-  const size_t scores = up256(static_cast<size_t>(s->batch) * s->n_kv_heads * n_blocks_max(s) * sizeof(float));
-  return std::max(total, scores);
+  return ready_words_offset(s) + up256(static_cast<size_t>(s->batch) * s->n_kv_heads * sizeof(int));
 }
 
 size_t tls_slab_bytes(const tls_shape *s) {
@@ -357,19 +364,19 @@ tls_status tls_token_score_topk(const tls_shape *s, const void *q, const void *s
 static tls_status select_step_impl(const tls_shape *s, const void *q, const void *meta, const void *slab,
                                    const int32_t *label_idx, const int32_t *seq_lens, int32_t *block_idx_out,
                                    int32_t *token_idx_out, float *block_score_out, float *token_score_out,
-                                   float *scratch, void *stream);
+                                   float *scratch, int **ready, int seq, void *stream);
 
 tls_status tls_select_step(const tls_shape *s, const void *q, const void *meta, const void *slab,
                            const int32_t *label_idx, const int32_t *seq_lens, int32_t *block_idx_out,
                            int32_t *token_idx_out, float *block_score_out, float *token_score_out, void *stream) {
   return select_step_impl(s, q, meta, slab, label_idx, seq_lens, block_idx_out, token_idx_out, block_score_out,
-                          token_score_out, nullptr, stream);
+                          token_score_out, nullptr, nullptr, 0, stream);
 }
 
 static tls_status select_step_impl(const tls_shape *s, const void *q, const void *meta, const void *slab,
                                    const int32_t *label_idx, const int32_t *seq_lens, int32_t *block_idx_out,
                                    int32_t *token_idx_out, float *block_score_out, float *token_score_out,
-                                   float *scratch, void *stream) {
+                                   float *scratch, int **ready, int seq, void *stream) {
   tls_status st = check_shape(s);
   if (st != TLS_OK) return st;
   if (s->batch == 0) return TLS_OK;
@@ -389,12 +396,18 @@ static tls_status select_step_impl(const tls_shape *s, const void *q, const void
                    s->n_kv_heads, s->d_qk, s->block_size, n_blocks_max(s), s->max_ctx, s->n_label, s->k_b, s->k_t,
                    s->kv_dtype, err, slab_scales(s, slab)};
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  // The readiness words (*ready, when given) are set by the select_step launch
+  // only; a path without it reports NULL back so that nothing waits on them.
+  t.ready = ready ? *ready : nullptr;
+  t.seq = seq;
   if (s->block_agg == 1) {
     st = agg_max_scores(s, a, block_score_out ? block_score_out : scratch, cs);
     if (st != TLS_OK) return st;
     if (a.from_scores)  // tensor-core scores: the cluster launch selects blocks, then tokens
       return cuda_status(tls::launch_select_step(a, t, cs), "select_step launch");
     // CUDA-core max-over-heads scores: the two separate launches
+    if (ready) *ready = nullptr;
+    t.ready = nullptr;
     st = cuda_status(tls::launch_block_select(a, cs), "block_select launch");
     if (st != TLS_OK) return st;
     return cuda_status(tls::launch_token_select(t, cs), "token_select launch");
@@ -416,7 +429,8 @@ static tls_status select_step_impl(const tls_shape *s, const void *q, const void
 
 static tls_status attn_common(const tls_shape *s, const void *q, const void *K, const void *V,
                               const int32_t *token_idx, const int32_t *slot_of_block, int32_t n_slots, void *out,
-                              float *lse_out, void *ws, size_t ws_bytes, void *stream, bool paged) {
+                              float *lse_out, void *ws, size_t ws_bytes, void *stream, bool paged,
+                              const int *ready = nullptr, int seq = 0) {
   tls_status st = check_shape(s);
   if (st != TLS_OK) return st;
   if (s->batch == 0) return TLS_OK;
@@ -447,6 +461,8 @@ static tls_status attn_common(const tls_shape *s, const void *q, const void *K, 
   a.part = reinterpret_cast<float *>(static_cast<char *>(ws) + w.part_off);
   a.err = tls::device_error_word();
   a.paged = paged;
+  a.ready = ready;
+  a.seq = seq;
   tls::AttnPlan p;
   if (!tls::attn_plan(a, &p)) return fail(TLS_ERR_UNSUPPORTED, "no attention plan for this shape");
   return cuda_status(tls::launch_attention(a, p, static_cast<cudaStream_t>(stream)), "attention launch");
@@ -554,12 +570,21 @@ tls_status tls_decode_step(const tls_shape *s, const void *q, const void *meta, 
   if (!need) return fail(TLS_ERR_UNSUPPORTED, "no workspace layout for this shape");
   if (!ws || ws_bytes < need || !aligned(ws, 256))
     return fail(TLS_ERR_WORKSPACE, "workspace too small or not 256-byte aligned (need %zu bytes)", need);
-  // the block scores may borrow the workspace: they are consumed by the
-  // selection launch before the attention writes its partials there
+  // The block scores may borrow the workspace: they are consumed by the
+  // selection launch before the attention writes its partials there.  When
+  // the attention is the warp-MMA kernel, the selection launch marks each
+  // group ready in the workspace's readiness words and lets the attention
+  // start early: its warps wait per group instead of for the whole grid.
+  tls::AttnArgs probe = attn_args(s);
+  tls::AttnPlan plan;
+  const bool overlap = tls::attn_plan(probe, &plan) && plan.impl == 2;
+  int *ready = overlap ? reinterpret_cast<int *>(static_cast<char *>(ws) + ready_words_offset(s)) : nullptr;
+  static std::atomic<int> g_seq{0};
+  const int seq = overlap ? (g_seq.fetch_add(1) & 0x3fffffff) + 1 : 0;
   st = select_step_impl(s, q, meta, slab, label_idx, seq_lens, block_idx_out, token_idx_out, block_score_out,
-                        token_score_out, static_cast<float *>(ws), stream);
+                        token_score_out, static_cast<float *>(ws), &ready, seq, stream);
   if (st != TLS_OK) return st;
-  return tls_sparse_attn_decode(s, q, K, V, token_idx_out, out, lse_out, ws, ws_bytes, stream);
+  return attn_common(s, q, K, V, token_idx_out, nullptr, 0, out, lse_out, ws, ws_bytes, stream, false, ready, seq);
 }
 
 tls_status tls_wait_event(void *event, int32_t timeout_ms) {

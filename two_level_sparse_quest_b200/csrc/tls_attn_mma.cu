@@ -50,7 +50,9 @@ __global__ void __launch_bounds__(MmaLayout<D, NS>::W * 32, 1) attn_mma_kernel(A
   long long *Off = reinterpret_cast<long long *>(wbase + NS * L::kStageBytes);  // [NS][kMT] byte offsets
   uint32_t *Mask = reinterpret_cast<uint32_t *>(Off + NS * kMT);                 // [NS] valid-token bits
 
-  grid_dependency_wait();
+  // With readiness words the selection launch before this one let it start
+  // early; each warp then waits for its groups (issue_next) instead of the grid.
+  if (!a.ready) grid_dependency_wait();
   const int gw = blockIdx.x * L::W + warp;
   const int t_begin = gw * p.tiles_per_warp;
   const int t_end = min(t_begin + p.tiles_per_warp, p.total_tiles);
@@ -69,6 +71,7 @@ __global__ void __launch_bounds__(MmaLayout<D, NS>::W * 32, 1) attn_mma_kernel(A
   const int unit0 = t_begin / p.tiles_per_group;
   int iss_t = t_begin, iss_group = unit0 / nhc, iss_hc = unit0 % nhc, iss_tile = t_begin % p.tiles_per_group,
       iss_st = 0;
+  int ready_group = -1;  // the last group whose readiness word this warp has seen
   auto issue_next = [&]() {
     const int t = iss_t, st = iss_st, tile = iss_tile, group = iss_group;
     if (++iss_tile == p.tiles_per_group) {
@@ -81,11 +84,25 @@ __global__ void __launch_bounds__(MmaLayout<D, NS>::W * 32, 1) attn_mma_kernel(A
     ++iss_t;
     if (++iss_st == NS) iss_st = 0;
     if (t < t_end) {
+      if (a.ready && group != ready_group) {  // bounded wait for the group's token ids
+        if (lane == 0) {
+          bool ok = false;
+          for (uint32_t i = 0; i < (1u << 22) && !ok; ++i) {
+            int v;
+            asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(a.ready + group) : "memory");
+            ok = v == a.seq;
+            if (!ok) __nanosleep(i < 16 ? 32 : 256);
+          }
+          if (!ok && a.err) atomicOr(a.err, kErrAttnWait);
+        }
+        __syncwarp();
+        ready_group = group;
+      }
       long long off = -1;
       if (lane < kMT) {
         const int j = tile * kMT + lane;
         if (j < a.k_t) {
-          const int tok = a.token_idx[static_cast<size_t>(group) * a.k_t + j];
+          const int tok = __ldcg(a.token_idx + static_cast<size_t>(group) * a.k_t + j);
           if (tok >= 0 && tok < a.max_ctx) {
             if constexpr (PAGED) {
               const int slot = a.slot_of_block[static_cast<size_t>(group) * a.n_blocks_max + tok / a.block_size];

@@ -112,6 +112,11 @@ struct TokenArgs {
   int batch, n_q_heads, n_kv_heads, d, block_size, n_blocks_max, max_ctx, n_label, k_b, k_t, dtype;
   int *err;           // the library's device error word
   const float *scales;  // int8 slab: [B*H_kv][r] channel scales; nullptr for a slab of the K dtype
+  // select_step only (nullable): per-group readiness words.  The launch resets
+  // its group's word, lets the dependent launch start early, and stores `seq`
+  // into it (release) once the group's token ids are written.
+  int *ready;
+  int seq;
 };
 // Token score and top-K_t in one launch (one thread-block cluster per group).
 cudaError_t launch_token_select(const TokenArgs &a, cudaStream_t st);
@@ -133,6 +138,11 @@ struct AttnArgs {
   int dtype, out_dtype, paged;
   float scale_log2;  // softmax_scale * log2(e)
   int num_sms;
+  // warp-MMA kernel only (nullable): per-group readiness words set by the
+  // selection launch before it (instead of waiting for that whole grid, each
+  // warp waits for its groups' words to equal seq).
+  const int *ready;
+  int seq;
 };
 // Partial-result layout chosen for a shape on a device; shared by the
 // workspace query and the launch so both agree.

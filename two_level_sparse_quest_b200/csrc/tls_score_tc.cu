@@ -98,7 +98,8 @@ static_assert(score_tc_smem(64, 18) <= 227 * 1024, "shared memory budget of the 
 
 // NP: padded heads (MMA N).  KR: 64-channel regions of K = 2 d.
 template <int NP, int KR>
-__global__ void __launch_bounds__(kSThreads, 1) block_scores_max_tc_kernel(BlockScoreArgs a, int n_items) {
+__global__ void __launch_bounds__(kSThreads, 1) block_scores_max_tc_kernel(BlockScoreArgs a, int n_items,
+                                                                          int items_per_cta) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char *smem =
       reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -111,8 +112,10 @@ __global__ void __launch_bounds__(kSThreads, 1) block_scores_max_tc_kernel(Block
   const int RB = 2 * d * 2;  // summary row bytes
   const int G = a.n_q_heads / a.n_kv_heads;
   const int tiles_per_group = (a.n_blocks_max + kSTile - 1) / kSTile;
-  // this CTA's work items: blockIdx.x, blockIdx.x + gridDim.x, ...
-  const int my_items = blockIdx.x < n_items ? (n_items - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  // this CTA's work items: a contiguous range, so that consecutive tiles
+  // mostly belong to the same group and share its B
+  const int item0 = blockIdx.x * items_per_cta;
+  const int my_items = max(0, min(items_per_cta, n_items - item0));
   if (my_items == 0) return;
 
   constexpr uint32_t kCols = NP <= 32 ? 32 : (NP <= 64 ? 64 : (NP <= 128 ? 128 : 256));
@@ -139,7 +142,7 @@ __global__ void __launch_bounds__(kSThreads, 1) block_scores_max_tc_kernel(Block
   // [64 r, 64 r + 64) of K; rows at or beyond the capacity are zero-filled.
   auto issue_region = [&](int step, int st) {
     const int it = step / KR, r = step % KR;
-    const int item = blockIdx.x + it * gridDim.x;
+    const int item = item0 + it;
     const int group = item / tiles_per_group, j0 = (item % tiles_per_group) * kSTile;
     const char *base = static_cast<const char *>(a.meta) + (static_cast<size_t>(group) * a.n_blocks_max) * RB;
     unsigned char *dst = ring + st * kSRegion;
@@ -152,22 +155,48 @@ __global__ void __launch_bounds__(kSThreads, 1) block_scores_max_tc_kernel(Block
       cp_async16(dst + s_sw(row, c), base + static_cast<size_t>(ok ? j : 0) * RB + r * 128 + c * 16, ok);
     }
   };
-  // B for a group: row h (< G) = [q_h^+ (d) ; q_h^- (d)] as bf16; rows G..NP-1 zero.
+  // B for a group: row h (< G) = [q_h^+ (d) ; q_h^- (d)] as bf16 (q^+ = max(q, 0),
+  // q^- = min(q, 0), taken from the sign bit of each bf16; -0 reads as 0).  The
+  // q rows are read as 16-byte chunks of 8 channels, kBLoads chunks in flight
+  // per thread; chunk c of row h lands in chunk c % 8 of region c / 8 (q^+)
+  // and of region (d / 64) + c / 8 (q^-).  Rows G .. NP-1 stay zero.
+  constexpr int kBLoads = 8;
   auto build_b = [&](int group) {
     const int b = group / a.n_kv_heads, g = group % a.n_kv_heads;
-    const uint16_t *q = static_cast<const uint16_t *>(a.q) + (static_cast<size_t>(b) * a.n_q_heads + g * G) * d;
-    for (int i = tid; i < NP * 2 * d; i += kSThreads) {
-      const int h = i / (2 * d), k = i % (2 * d);
-      uint16_t v = 0;
-      if (h < G) {
-        const uint16_t x = q[h * d + (k < d ? k : k - d)];
-        const bool neg = (x & 0x8000u) != 0;
-        v = (k < d) ? (neg ? 0 : x) : (neg ? x : 0);  // q^+ = max(q, 0), q^- = min(q, 0); -0 reads as 0
+    const uint4 *q4 = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(a.q) +
+                                                      (static_cast<size_t>(b) * a.n_q_heads + g * G) * d);
+    const int cpr = d / 8, n = G * cpr, half = d / 64;
+    for (int base = 0; base < n; base += kSThreads * kBLoads) {
+      uint4 v[kBLoads];
+#pragma unroll
+      for (int u = 0; u < kBLoads; ++u) {
+        const int idx = base + u * kSThreads + tid;
+        v[u] = idx < n ? q4[idx] : make_uint4(0, 0, 0, 0);
       }
-      const int r = k >> 6, col = k & 63;
-      *reinterpret_cast<uint16_t *>(bmat + r * NP * 128 + s_sw(h, col >> 3) + (col & 7) * 2) = v;
+#pragma unroll
+      for (int u = 0; u < kBLoads; ++u) {
+        const int idx = base + u * kSThreads + tid;
+        if (idx < n) {
+          const int h = idx / cpr, c = idx % cpr;
+          uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w}, pw[4], nw[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t m = ((w[i] >> 15) & 0x00010001u) * 0xFFFFu;  // 0xFFFF in each negative half
+            nw[i] = w[i] & m;
+            pw[i] = w[i] & ~m;
+          }
+          *reinterpret_cast<uint4 *>(bmat + (c >> 3) * NP * 128 + s_sw(h, c & 7)) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+          *reinterpret_cast<uint4 *>(bmat + (half + (c >> 3)) * NP * 128 + s_sw(h, c & 7)) =
+              make_uint4(nw[0], nw[1], nw[2], nw[3]);
+        }
+      }
     }
   };
+  // rows G .. NP-1 of every region: zero for the whole launch
+  for (int i = tid; i < KR * NP * 8; i += kSThreads) {
+    const int r = i / (NP * 8), h = (i / 8) % NP, c = i % 8;
+    if (h >= G) *reinterpret_cast<uint4 *>(bmat + r * NP * 128 + s_sw(h, c)) = make_uint4(0, 0, 0, 0);
+  }
 
   const int n_steps = my_items * KR;
   int cur_group = -1;
@@ -183,7 +212,7 @@ __global__ void __launch_bounds__(kSThreads, 1) block_scores_max_tc_kernel(Block
   for (int step = 0; step < n_steps && !failed; ++step) {
     const int st = step % kSStages;
     const int it = step / KR, r = step % KR;
-    const int item = blockIdx.x + it * gridDim.x;
+    const int item = item0 + it;
     const int group = item / tiles_per_group;
     // the stage that region step + kSStages - 1 reuses held region step - 1:
     // its MMA must be complete before the copies overwrite it
@@ -259,8 +288,9 @@ cudaError_t run_score_tc(const BlockScoreArgs &a, int num_sms, cudaStream_t st) 
   }
   const long long items = static_cast<long long>(a.batch) * a.n_kv_heads * ((a.n_blocks_max + kSTile - 1) / kSTile);
   if (items <= 0 || items > (1LL << 30)) return cudaErrorInvalidValue;
-  const int grid = static_cast<int>(std::min<long long>(num_sms, items));
-  return launch_pdl(kern, dim3(grid), dim3(kSThreads), static_cast<size_t>(smem), st, a, static_cast<int>(items));
+  const int per = static_cast<int>((items + num_sms - 1) / num_sms);  // contiguous items per CTA
+  const int grid = static_cast<int>((items + per - 1) / per);
+  return launch_pdl(kern, dim3(grid), dim3(kSThreads), static_cast<size_t>(smem), st, a, static_cast<int>(items), per);
 }
 
 template <int KR>

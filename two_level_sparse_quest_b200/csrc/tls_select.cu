@@ -414,6 +414,14 @@ __global__ void __launch_bounds__(kThreads, NCH > 32 ? 2 : token_min_blocks<RCH,
     ST.hist[threadIdx.x] = 0;
   }
   grid_dependency_wait();
+  if (t.ready) {  // the attention after this launch waits per group on these words, not on the grid
+    if (rank == 0 && threadIdx.x == 0) {
+      t.ready[group] = 0;
+      __threadfence();
+    }
+    __syncthreads();
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  }
   const int b = group / a.n_kv_heads;
   const int sq = min(max(a.seq_lens[b], 0), a.max_ctx);
   const int nb = (sq + a.block_size - 1) / a.block_size;
@@ -446,6 +454,13 @@ __global__ void __launch_bounds__(kThreads, NCH > 32 ? 2 : token_min_blocks<RCH,
         return blk[jb - jb0] * bs + (j - jb * bs);
       },
       ST, t.err, /*entry_wait=*/false);
+  if (t.ready) {  // every CTA's token ids are written: the group is ready for its attention
+    __threadfence();
+    cluster_arrive_release();
+    cluster_wait();
+    if (rank == 0 && threadIdx.x == 0)
+      asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(t.ready + group), "r"(t.seq) : "memory");
+  }
 }
 
 // ---------------------------------------------------------------- launchers
