@@ -110,7 +110,7 @@ TLS_API const char *tls_last_error(void);
 /* Bytes of device workspace that tls_sparse_attn_decode(_paged) and
  * tls_decode_step need for this shape on the current device (the split-KV
  * partials; tls_decode_step also keeps the step's block scores there before
- * the attention runs).  Calls that run
+ * the attention runs, and one readiness word per group after them).  Calls that run
  * concurrently need separate buffers.  The selection stages take a workspace
  * argument too but use none (their keys stay in on-chip memory); they accept
  * NULL.  Returns 0 for an invalid shape (see tls_last_error). */
@@ -239,7 +239,14 @@ TLS_API tls_status tls_select_step(const tls_shape *s, const void *q, const void
  *   out, lse_out                         as in tls_sparse_attn_decode (lse may be NULL)
  *   block_score_out, token_score_out     as in tls_select_step, or NULL
  *   ws, ws_bytes                         as in tls_sparse_attn_decode (checked
- *                                        before anything is enqueued) */
+ *                                        before anything is enqueued)
+ * When the attention is the warp-MMA kernel (bf16 GQA, d in {64, 128}), the
+ * two launches overlap: the selection launch resets one readiness word per
+ * group in the workspace, lets the attention launch start early and marks a
+ * group ready once its token ids are written; the attention's warps wait per
+ * group (bounded: a wait that gives up sets bit 1 of tls_device_error) rather
+ * than for the whole selection grid.  Calls on one workspace must not overlap
+ * on the GPU. */
 TLS_API tls_status tls_decode_step(const tls_shape *s, const void *q, const void *meta, const void *slab,
                                    const int32_t *label_idx, const int32_t *seq_lens, const void *K, const void *V,
                                    int32_t *block_idx_out, int32_t *token_idx_out, void *out, float *lse_out,
