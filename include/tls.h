@@ -110,7 +110,8 @@ TLS_API const char *tls_last_error(void);
 /* Bytes of device workspace that tls_sparse_attn_decode(_paged) and
  * tls_decode_step need for this shape on the current device (the split-KV
  * partials; tls_decode_step also keeps the step's block scores there before
- * the attention runs, and one readiness word per group after them).  Calls that run
+ * the attention runs, and after them one readiness word per group and the
+ * groups' folded queries [Q+; Q-], 2 d_qk fp32 each).  Calls that run
  * concurrently need separate buffers.  The selection stages take a workspace
  * argument too but use none (their keys stay in on-chip memory); they accept
  * NULL.  Returns 0 for an invalid shape (see tls_last_error). */
@@ -219,7 +220,9 @@ TLS_API tls_status tls_token_score_topk(const tls_shape *s, const void *q, const
  * summary, at most 16 query heads per KV head and block_score_out given, the
  * block scores are first computed by a grid over all SMs into block_score_out
  * and the clusters select from them (two launches, same bits): one cluster
- * per group alone cannot keep HBM busy.
+ * per group alone cannot keep HBM busy.  Each CTA of a group's cluster then
+ * selects the K_b blocks itself from the group's scores (at most 4096 blocks;
+ * above that the cluster selects them together).
  * Arguments as in those two calls; block_idx_out is written and then read
  * back by the same launch.  block_score_out / token_score_out may be NULL.
  * block_agg 1 with bf16 keys and more than 8 heads per group (or the latent
@@ -230,7 +233,12 @@ TLS_API tls_status tls_select_step(const tls_shape *s, const void *q, const void
                                    void *stream);
 
 /* Stages 1-5 in one call: tls_select_step, then tls_sparse_attn_decode on its
- * token ids, for callers that want the whole decode step.
+ * token ids, for callers that want the whole decode step.  Its two-phase
+ * selection (few groups, as in tls_select_step, the block scores in the
+ * workspace unless block_score_out is given) also serves groups of more than
+ * 16 query heads: a small launch first folds each group's queries once into
+ * the workspace, which the phase-1 grid reads (the same bits as the fold each
+ * CTA does otherwise).
  * gist.science (de) section 2.A and (es) section 2.A (the five stages); the
  * two calls above give the definitions.  Arguments:
  *   q, meta, slab, label_idx, seq_lens   as in tls_select_step

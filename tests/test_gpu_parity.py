@@ -46,6 +46,14 @@ SMALL = {
     "block_size_16_odd_ctx": (W.WORKLOADS["gqa48k_bf16"].with_(block_size=16, ctx=1999, k_b=40, k_t=333), None),
     "mla_small": (W.WORKLOADS["mla64k_b4_bf16"].with_(batch=2, ctx=4096, k_b=16, k_t=300, n_needles=4),
                   [4096, 3000]),
+    # latent shapes with 16 and 32 heads, and a batch whose CTA ranges of
+    # 32-token tiles cross group boundaries (35 tiles per group, 2 per CTA)
+    "mla_g16": (W.WORKLOADS["mla64k_b4_bf16"].with_(batch=3, n_q_heads=16, ctx=4096, k_b=16, k_t=300, n_needles=4),
+                [4096, 2100, 0]),
+    "mla_g32": (W.WORKLOADS["mla64k_b4_bf16"].with_(batch=2, n_q_heads=32, ctx=4096, k_b=16, k_t=300, n_needles=4),
+                [3001, 4096]),
+    "mla_ranges_cross_groups": (W.WORKLOADS["mla64k_b4_bf16"].with_(batch=6, ctx=8192, k_b=24, k_t=1100, n_needles=8),
+                                [8192, 5000, 33, 8192, 1, 7000]),
     # shape sweep: MHA (one query head per KV head) and MQA (one KV head for
     # 16, 32 or 64 query heads: units of 16 heads on the warp-MMA kernel)
     "mha_h16": (W.WORKLOADS["gqa48k_bf16"].with_(n_q_heads=16, n_kv_heads=16, ctx=2048, k_b=16, k_t=200), None),
@@ -65,6 +73,24 @@ def test_small_parity(name):
     w, sl = SMALL[name]
     res = P().full_stage_parity(w, seq_lens=sl, name=name)
     assert res["chained_groups_identical"] >= 0
+
+
+def sharpened(inp, factor):
+    """The same inputs with every bf16 query multiplied by a power of two
+    (exact): the block and token rankings do not change, the softmax becomes
+    sharper, and a head's running max grows by many log2 units across tiles."""
+    q = (inp.q.astype(np.uint32) << 16).view(np.float32) * np.float32(factor)
+    inp.q = (q.view(np.uint32) >> 16).astype(np.uint16)
+    return inp
+
+
+@pytest.mark.parametrize("name,factor", [("mla_ranges_cross_groups", 16.0), ("mla_small", 64.0)])
+def test_latent_attention_sharp_softmax(name, factor):
+    """Large score spreads: the latent kernel's reference max moves and the
+    running output is rescaled inside a CTA's range."""
+    w, sl = SMALL[name]
+    inp = sharpened(W.make_decode_inputs(w, seq_lens=sl), factor)
+    P().full_stage_parity(w, inp=inp, name=f"{name}:x{factor:g}")
 
 
 def test_bf16_output_parity():
@@ -159,18 +185,20 @@ def test_full_size_parity(name):
     assert res["token_swaps"] <= max(1, res["groups"] // 8)
 
 
-@pytest.mark.parametrize("impl", ["cuda_core", "tensor_core"])
+@pytest.mark.parametrize("impl", ["cuda_core", "tensor_core", "warp_mma"])
 def test_alternative_attention_kernels_parity(impl):
     """The attention kernels that TLS_ATTN_IMPL selects instead of the default
     (read once per process, so each runs in a child process): the CUDA-core
-    kernel for GQA bf16 and latent shapes, the tcgen05 kernel for GQA bf16."""
+    kernel for GQA bf16 and latent shapes, the tcgen05 kernel for GQA bf16,
+    the warp-MMA latent kernel for latent shapes."""
     import os
     import subprocess
     import sys
 
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    cases = (["gqa_bf16_small", "gqa_bf16_g8", "mla_small", "mqa_g32", "mqa_g64_d64"] if impl == "cuda_core"
-             else ["gqa_bf16_small", "gqa_bf16_g8"])
+    cases = {"cuda_core": ["gqa_bf16_small", "gqa_bf16_g8", "mla_small", "mqa_g32", "mqa_g64_d64"],
+             "tensor_core": ["gqa_bf16_small", "gqa_bf16_g8"],
+             "warp_mma": ["mla_small", "mla_g16", "mla_g32"]}[impl]
     code = (
         "import sys; sys.path.insert(0, %r)\n"
         "from tests import test_gpu_parity as t, _parity as P\n"

@@ -19,7 +19,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OUT = os.path.join(PKG, "libtls.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
-SOURCES = ["tls_api.cu", "tls_meta.cu", "tls_select.cu", "tls_attn.cu", "tls_offload.cu", "tls_noalloc.cu", "tls_attn_tc.cu", "tls_attn_mma.cu", "tls_attn_mla.cu", "tls_score_tc.cu"]
+SOURCES = ["tls_api.cu", "tls_meta.cu", "tls_select.cu", "tls_attn.cu", "tls_offload.cu", "tls_noalloc.cu", "tls_attn_tc.cu", "tls_attn_mma.cu", "tls_attn_mla.cu", "tls_attn_mla_tc.cu", "tls_score_tc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", INCLUDE, "-I", CSRC]

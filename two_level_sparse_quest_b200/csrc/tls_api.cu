@@ -184,6 +184,12 @@ size_t ready_words_offset(const tls_shape *s) {
   return up256(std::max(body, scores));
 }
 
+// Then the folded queries of the two-phase selection ([B*H_kv][2 d] fp32) at
+// this offset.
+size_t fold_offset(const tls_shape *s) {
+  return ready_words_offset(s) + up256(static_cast<size_t>(s->batch) * s->n_kv_heads * sizeof(int));
+}
+
 // The library's device error word: one int per GPU, zero until a kernel's
 // bounded wait gives up (bits kErrAttnWait, kErrSelectWait).
 __device__ int g_device_error;
@@ -233,7 +239,7 @@ size_t tls_workspace_size(const tls_shape *s) {
     fail(TLS_ERR_UNSUPPORTED, "no attention plan for this shape");
     return 0;
   }
-  return ready_words_offset(s) + up256(static_cast<size_t>(s->batch) * s->n_kv_heads * sizeof(int));
+  return fold_offset(s) + up256(static_cast<size_t>(s->batch) * s->n_kv_heads * 2 * s->d_qk * sizeof(float));
 }
 
 size_t tls_slab_bytes(const tls_shape *s) {
@@ -364,19 +370,19 @@ tls_status tls_token_score_topk(const tls_shape *s, const void *q, const void *s
 static tls_status select_step_impl(const tls_shape *s, const void *q, const void *meta, const void *slab,
                                    const int32_t *label_idx, const int32_t *seq_lens, int32_t *block_idx_out,
                                    int32_t *token_idx_out, float *block_score_out, float *token_score_out,
-                                   float *scratch, int **ready, int seq, void *stream);
+                                   float *scratch, float *qfold, int **ready, int seq, void *stream);
 
 tls_status tls_select_step(const tls_shape *s, const void *q, const void *meta, const void *slab,
                            const int32_t *label_idx, const int32_t *seq_lens, int32_t *block_idx_out,
                            int32_t *token_idx_out, float *block_score_out, float *token_score_out, void *stream) {
   return select_step_impl(s, q, meta, slab, label_idx, seq_lens, block_idx_out, token_idx_out, block_score_out,
-                          token_score_out, nullptr, nullptr, 0, stream);
+                          token_score_out, nullptr, nullptr, nullptr, 0, stream);
 }
 
 static tls_status select_step_impl(const tls_shape *s, const void *q, const void *meta, const void *slab,
                                    const int32_t *label_idx, const int32_t *seq_lens, int32_t *block_idx_out,
                                    int32_t *token_idx_out, float *block_score_out, float *token_score_out,
-                                   float *scratch, int **ready, int seq, void *stream) {
+                                   float *scratch, float *qfold, int **ready, int seq, void *stream) {
   tls_status st = check_shape(s);
   if (st != TLS_OK) return st;
   if (s->batch == 0) return TLS_OK;
@@ -418,8 +424,13 @@ static tls_status select_step_impl(const tls_shape *s, const void *q, const void
   const size_t summary_bytes = static_cast<size_t>(s->batch) * s->n_kv_heads * n_blocks_max(s) * 2 * s->d_qk *
                                (s->kv_dtype == TLS_BF16 ? 2 : 4);
   if (scores && tls::select_two_phase(s->batch * s->n_kv_heads, s->n_q_heads / s->n_kv_heads, device_sms(),
-                                      summary_bytes)) {
+                                      summary_bytes, qfold != nullptr)) {
     a.scores = scores;
+    if (qfold) {  // the queries folded once per group, not by every phase-1 CTA
+      a.qfold = qfold;
+      st = cuda_status(tls::launch_query_fold(a, cs), "query_fold launch");
+      if (st != TLS_OK) return st;
+    }
     st = cuda_status(tls::launch_block_scores(a, device_sms(), cs), "block_scores launch");
     if (st != TLS_OK) return st;
     a.from_scores = 1;
@@ -582,7 +593,8 @@ tls_status tls_decode_step(const tls_shape *s, const void *q, const void *meta, 
   static std::atomic<int> g_seq{0};
   const int seq = overlap ? (g_seq.fetch_add(1) & 0x3fffffff) + 1 : 0;
   st = select_step_impl(s, q, meta, slab, label_idx, seq_lens, block_idx_out, token_idx_out, block_score_out,
-                        token_score_out, static_cast<float *>(ws), &ready, seq, stream);
+                        token_score_out, static_cast<float *>(ws),
+                        reinterpret_cast<float *>(static_cast<char *>(ws) + fold_offset(s)), &ready, seq, stream);
   if (st != TLS_OK) return st;
   return attn_common(s, q, K, V, token_idx_out, nullptr, 0, out, lse_out, ws, ws_bytes, stream, false, ready, seq);
 }

@@ -416,18 +416,21 @@ cudaError_t dispatch_gqa(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) 
 }  // namespace
 
 // Kernel choice.  bf16 GQA shapes run the warp-MMA kernel (tls_attn_mma.cu)
-// and latent shapes with 16, 32 or 64 heads the warp-MMA latent kernel
-// (tls_attn_mla.cu) by default; TLS_ATTN_IMPL=cuda_core selects this file's
-// CUDA-core kernel for both, TLS_ATTN_IMPL=tensor_core the tcgen05 kernel
-// (bf16 GQA, d = 128).  The variable is read once per process.  fp32 shapes
-// and other latent head counts always run the CUDA-core kernel.
-enum ImplChoice { kImplDefault = 0, kImplCudaCore = 1, kImplTcgen05 = 2 };
+// and latent shapes with up to 64 heads per group the tcgen05 latent kernel
+// (tls_attn_mla_tc.cu) by default.  TLS_ATTN_IMPL=cuda_core selects this
+// file's CUDA-core kernel for both, TLS_ATTN_IMPL=tensor_core the tcgen05
+// kernel for bf16 GQA (d = 128), TLS_ATTN_IMPL=warp_mma the warp-MMA latent
+// kernel (tls_attn_mla.cu; 16, 32 or 64 heads).  The variable is read once
+// per process.  fp32 shapes and other latent head counts always run the
+// CUDA-core kernel.
+enum ImplChoice { kImplDefault = 0, kImplCudaCore = 1, kImplTcgen05 = 2, kImplWarpMma = 3 };
 static int impl_choice() {
   static int choice = -1;
   if (choice < 0) {
     const char *e = getenv("TLS_ATTN_IMPL");
     if (e && strcmp(e, "tensor_core") == 0) choice = kImplTcgen05;
     else if (e && strcmp(e, "cuda_core") == 0) choice = kImplCudaCore;
+    else if (e && strcmp(e, "warp_mma") == 0) choice = kImplWarpMma;
     else choice = kImplDefault;
   }
   return choice;
@@ -439,17 +442,19 @@ bool attn_plan(const AttnArgs &a, AttnPlan *p) {
     p->impl = 1;
     return attn_tc_plan(a, p);
   }
-  if (choice == kImplDefault && attn_mla_supported(a)) {
+  const bool mla_tc = (choice == kImplDefault || choice == kImplTcgen05) && attn_mla_tc_supported(a);
+  if (mla_tc || (choice == kImplWarpMma && attn_mla_supported(a))) {
     // latent attention on the tensor cores: a unit is a whole group (all G
-    // heads), a piece is one CTA's contiguous range of 16-token tiles
+    // heads), a piece is one CTA's contiguous range of tiles
     const int G = a.n_q_heads / a.n_kv_heads;
-    p->impl = 3;
-    p->warps_per_cta = 8;
-    p->tokens_per_tile = 16;
+    const int tt = mla_tc ? attn_mla_tc_tokens_per_tile() : 16;
+    p->impl = mla_tc ? 5 : 3;
+    p->warps_per_cta = mla_tc ? 4 : 8;
+    p->tokens_per_tile = tt;
     p->head_chunk = G;
     p->n_head_chunks = 1;
     const long long units = static_cast<long long>(a.batch) * a.n_kv_heads;
-    p->tiles_per_group = (a.k_t + 15) / 16;
+    p->tiles_per_group = (a.k_t + tt - 1) / tt;
     const long long total = units * p->tiles_per_group;
     if (total <= 0 || total > (1LL << 30)) return false;
     p->total_tiles = static_cast<int>(total);
@@ -492,6 +497,7 @@ static cudaError_t launch_split(const AttnArgs &a, const AttnPlan &p, cudaStream
   if (p.impl == 1) return launch_attention_tc(a, p, st);
   if (p.impl == 2) return launch_attention_mma(a, p, st);
   if (p.impl == 3) return launch_attention_mla(a, p, st);
+  if (p.impl == 5) return launch_attention_mla_tc(a, p, st);
   if (a.v_is_k_prefix) return run_attention<BF16, 576, 512, 4, true, false, kStages>(a, p, st);
   if (a.dtype == 1) {
     if (a.d_qk == 128) return a.paged ? dispatch_gqa<BF16, 128, true>(a, p, st) : dispatch_gqa<BF16, 128, false>(a, p, st);
@@ -503,8 +509,12 @@ static cudaError_t launch_split(const AttnArgs &a, const AttnPlan &p, cudaStream
 
 cudaError_t launch_attention_merge(const AttnArgs &a, const AttnPlan &p, cudaStream_t st) {
   if (a.v_is_k_prefix) {
-    if (p.impl == 3) {
+    if (p.impl == 3 || p.impl == 5) {
       switch (p.head_chunk) {
+        case 1: return run_merge<512, 1>(a, p, st);
+        case 2: return run_merge<512, 2>(a, p, st);
+        case 4: return run_merge<512, 4>(a, p, st);
+        case 8: return run_merge<512, 8>(a, p, st);
         case 16: return run_merge<512, 16>(a, p, st);
         case 32: return run_merge<512, 32>(a, p, st);
         case 64: return run_merge<512, 64>(a, p, st);

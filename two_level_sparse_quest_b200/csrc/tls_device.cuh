@@ -431,6 +431,73 @@ __device__ void ordered_compact(const uint32_t *keys, int n, SelectResult r, int
   }
 }
 
+// The same selection by one CTA over keys[0..n) in its own shared memory
+// (n <= CAP): four radix passes of 8 bits over a shared-memory histogram, then
+// the index-ordered compaction into out[0..k) (ascending ids; the caller pads).
+// Returns k (the wanted count clamped to the valid keys).  Every thread of the
+// CTA calls it; hist must hold kCBins ints, bc 4 ints, sh 33 ints.
+template <int NT, int CAP, typename IdOf>
+__device__ int cta_topk(const uint32_t *keys, int n, int k_req, int32_t *out, IdOf id_of, int *hist, int *bc,
+                        int *sh) {
+  static_assert(NT >= kCBins && NT % 32 == 0, "one histogram bin per thread");
+  const int tid = threadIdx.x, lane = tid & 31;
+  uint32_t prefix = 0;
+  int krem = 0, k = 0;
+  __syncthreads();  // the keys are complete and nothing still adds to hist
+#pragma unroll 1
+  for (int p = 0; p < 4; ++p) {
+    const int shift = 24 - 8 * p;
+    if (tid < kCBins) hist[tid] = 0;
+    __syncthreads();  // the previous pass's decision is read
+    const uint32_t want = p == 0 ? 0u : prefix >> (shift + 8);
+    for (int i = tid; i < n; i += NT) {
+      const uint32_t key = keys[i];
+      if (key != 0u && (p == 0 || (key >> (shift + 8)) == want)) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    }
+    __syncthreads();
+    if (tid < 32) {  // lane l owns bins 255-8l .. 248-8l, from the top
+      const int top = kCBins - 1 - 8 * lane;
+      int cnt[8], sum = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        cnt[j] = hist[top - j];
+        sum += cnt[j];
+      }
+      const int incl = warp_incl_scan(sum);
+      int kr = krem;
+      if (p == 0) kr = min(k_req, __shfl_sync(0xffffffffu, incl, 31));  // valid keys
+      int acc = incl - sum;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (acc < kr && acc + cnt[j] >= kr) {  // exactly one (lane, bin) satisfies this
+          bc[0] = top - j;
+          bc[1] = acc;
+          bc[3] = cnt[j];
+        }
+        acc += cnt[j];
+      }
+      if (p == 0 && lane == 0) bc[2] = kr;
+    }
+    __syncthreads();
+    if (p == 0) {
+      k = bc[2];
+      krem = k;
+      if (k <= 0) break;  // no valid key
+    }
+    krem -= bc[1];
+    prefix |= static_cast<uint32_t>(bc[0]) << shift;
+    if (krem == bc[3] && prefix != 0u) {  // exact fit: every key of the bin is kept
+      prefix -= 1u;
+      krem = 0;
+      break;
+    }
+  }
+  if (k > 0)
+    ordered_compact<NT, CAP>(keys, n, SelectResult{prefix, krem}, k, out, id_of, sh, [](int) { return 0; });
+  __syncthreads();
+  return k;
+}
+
 // The whole selection for one cluster (steps 2-3; step 1 done by the caller
 // into S.hist).  keys[0..n): this CTA's slice, n <= CAP; k_req: wanted count
 // (clamped to the number of valid keys of the group); out[0..cap): ids in

@@ -86,15 +86,20 @@ struct BlockScoreArgs {
   int *err;           // the library's device error word
   int agg;            // 0: sum of the heads' bounds, 1: their max
   int from_scores;    // 1: scores already hold the step's block scores (the cluster only selects)
+  float *qfold;       // [B*H_kv][2 d] folded queries [Q+; Q-] (written by launch_query_fold), or null
 };
 // Block score and top-K_b in one launch (one thread-block cluster per group).
 cudaError_t launch_block_select(const BlockScoreArgs &a, cudaStream_t st);
 // Whether the two-phase selection pays off for this many groups on this
 // device: the block summary is then streamed by a grid over all SMs into
 // a.scores first, and the clusters select from those scores.
-bool select_two_phase(int groups, int heads_per_group, int num_sms, size_t summary_bytes);
-// Phase 1 of the two-phase selection: every group's block scores into a.scores.
+bool select_two_phase(int groups, int heads_per_group, int num_sms, size_t summary_bytes, bool folded_queries);
+// Phase 1 of the two-phase selection: every group's block scores into a.scores
+// (from a.qfold when set, else every CTA folds its groups' queries itself).
 cudaError_t launch_block_scores(const BlockScoreArgs &a, int num_sms, cudaStream_t st);
+// [Q+; Q-] of every group into a.qfold, once per group, with the arithmetic
+// of the in-kernel fold (so the scores are the same bits either way).
+cudaError_t launch_query_fold(const BlockScoreArgs &a, cudaStream_t st);
 // The max-over-heads block scores (block_agg 1) of every group into a.scores,
 // as a tcgen05 GEMM [blocks x 2d] . [2d x heads] with a row maximum (bf16,
 // d in {64, 128, 576}, up to 64 heads per group).
@@ -147,8 +152,8 @@ struct AttnArgs {
 // Partial-result layout chosen for a shape on a device; shared by the
 // workspace query and the launch so both agree.
 struct AttnPlan {
-  int impl;  // 0: CUDA-core kernel, 1: tcgen05 kernel, 2: warp-MMA GQA kernel, 3: warp-MMA latent kernel
-             // (for 1 and 3 tiles_per_warp counts tiles per CTA)
+  int impl;  // 0: CUDA-core kernel, 1: tcgen05 kernel, 2: warp-MMA GQA kernel, 3: warp-MMA latent kernel,
+             // 5: tcgen05 latent kernel (for 1, 3 and 5 tiles_per_warp counts tiles per CTA)
   int warps_per_cta, tokens_per_tile, head_chunk, n_head_chunks;
   int tiles_per_group, total_tiles, grid, tiles_per_warp, max_pieces;
   size_t part_floats;  // floats of workspace for partials
@@ -158,6 +163,10 @@ cudaError_t launch_attention(const AttnArgs &a, const AttnPlan &p, cudaStream_t 
 // tensor-core (tcgen05) attention for GQA bf16 d = 128
 bool attn_mla_supported(const AttnArgs &a);
 cudaError_t launch_attention_mla(const AttnArgs &a, const AttnPlan &p, cudaStream_t st);
+// tcgen05 latent attention (bf16, d 576 / 512, up to 64 heads per group)
+bool attn_mla_tc_supported(const AttnArgs &a);
+int attn_mla_tc_tokens_per_tile();
+cudaError_t launch_attention_mla_tc(const AttnArgs &a, const AttnPlan &p, cudaStream_t st);
 bool attn_mma_supported(const AttnArgs &a);
 int attn_mma_warps(const AttnArgs &a);
 // Heads per unit of the warp-MMA kernel: the group, or 16 for larger groups.

@@ -39,13 +39,106 @@ constexpr int kClusterSize = 8;  // CTAs per group (portable cluster size)
 constexpr int kSliceCap = kMaxSelectKeys / kClusterSize;  // keys per CTA
 constexpr int kThreads = 256;
 
+// ---------------------------------------------------------------- query folds
+// Parts of a fold over the G heads of a group: the largest power of two P <=
+// G with P * items <= kThreads (and P <= 32), so that the P threads of an
+// item are consecutive lanes of one warp.
+__device__ __forceinline__ int fold_parts(int G, int items) {
+  int P = 1;
+  while (2 * P <= G && 2 * P <= 32 && 2 * P * items <= kThreads) P *= 2;
+  return P;
+}
+
+// Adds v of the P lanes of this item (lanes part 0 .. P-1, consecutive), in
+// part order, starting from 0: every lane of the warp calls it.
+__device__ __forceinline__ float fold_lanes(float v, int P) {
+  const int lane = threadIdx.x & 31, first = lane & ~(P - 1);
+  float sum = 0.f;
+  for (int k = 0; k < P; ++k) sum += __shfl_sync(0xffffffffu, v, first + k);
+  return sum;
+}
+
+// qpm = [Q+; Q-] (2 d floats of shared memory) of the G heads of query rows
+// row0 .. row0 + G - 1: Q+_i = sum_h max(q_{h,i}, 0), Q-_i = sum_h min(q_{h,i}, 0)
+// (gist.science (de) section 2.A "Stufe 1": the per-head bounds summed over
+// the heads that share the KV head).  All threads of the CTA call it.  The
+// G x d block is read as 16-byte chunks: thread t takes chunk column t / P and
+// the heads of part t % P (consecutive heads, 8 loads in flight); the P part
+// sums are then added in part order.  With P = G (small groups) the sums are
+// the sequential sums over the heads.  FB: loads in flight per thread.
+template <typename E, int FB>
+__device__ __forceinline__ void fold_group_query(const void *q, size_t row0, int G, int d, float *qpm) {
+  constexpr int EPC = E::kEPC;
+  const int NC = d / EPC;
+  const int P = fold_parts(G, NC);
+  const int HP = (G + P - 1) / P;
+  for (int base = 0; base < NC * P; base += kThreads) {  // one pass unless NC > kThreads
+    const int t = base + static_cast<int>(threadIdx.x);
+    const int c = t / P, part = t % P;
+    float pos[EPC], neg[EPC];
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) pos[e] = neg[e] = 0.f;
+    if (c < NC) {
+      const uint4 *src = static_cast<const uint4 *>(q) + row0 * NC + c;
+      const int h0 = part * HP, h1 = min(G, h0 + HP);
+      for (int hb = h0; hb < h1; hb += FB) {
+        uint4 v[FB];
+#pragma unroll
+        for (int u = 0; u < FB; ++u) v[u] = hb + u < h1 ? __ldg(src + static_cast<size_t>(hb + u) * NC) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int u = 0; u < FB; ++u) {
+          if (hb + u < h1) {
+            float f[EPC];
+            chunk_to_f32<E>(v[u], f);
+#pragma unroll
+            for (int e = 0; e < EPC; ++e) {
+              pos[e] += fmaxf(f[e], 0.f);
+              neg[e] += fminf(f[e], 0.f);
+            }
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < EPC; ++e) {
+      const float sp = fold_lanes(pos[e], P), sn = fold_lanes(neg[e], P);
+      if (c < NC && part == 0) {
+        qpm[c * EPC + e] = sp;
+        qpm[d + c * EPC + e] = sn;
+      }
+    }
+  }
+}
+
+// The fold every path uses (so that every path's block scores are the same
+// bits), by the summary row's 16-byte chunks NCH: for d <= 128 (NCH <= 64)
+// thread i sums channel i over the heads in order (few heads, short rows:
+// this is the cheapest), for the latent rows the parallel fold above.
+template <typename E, int NCH, int FB>
+__device__ __forceinline__ void fold_query(const void *q, size_t row0, int G, int d, float *qpm) {
+  if constexpr (NCH > 64) {
+    fold_group_query<E, FB>(q, row0, G, d, qpm);
+  } else {
+    for (int i = threadIdx.x; i < d; i += kThreads) {
+      float pos = 0.f, neg = 0.f;
+      for (int hh = 0; hh < G; ++hh) {
+        const float x = load_elem<E>(q, (row0 + hh) * d + i);
+        pos += fmaxf(x, 0.f);
+        neg += fminf(x, 0.f);
+      }
+      qpm[i] = pos;
+      qpm[d + i] = neg;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- stage 1 body
 // After the grid dependency wait: folds the group's query into qpm = [Q+; Q-]
 // and scores summary rows [r0, r1) into keys[row - r0] and hist (top key
 // byte).  NCH: 16-byte chunks per summary row (2 * d * bytes / 16).  The first
 // rows' loads are issued before the head fold so that the query reads
 // overlap them.
-template <typename E, int NCH, bool KEYS = true>
+template <typename E, int NCH, bool KEYS = true, bool QFOLD = false>
 __device__ __forceinline__ void score_blocks(const BlockScoreArgs &a, int group, int nb, int r0, int r1, float *qpm,
                                              uint32_t *keys, int *hist) {
   constexpr int EPC = E::kEPC;
@@ -78,15 +171,11 @@ __device__ __forceinline__ void score_blocks(const BlockScoreArgs &a, int group,
   uint4 v[U][CPL];
   int rb = r0 + warp * RPW;
   load_rows(rb, v);  // in flight while the query is folded
-  for (int i = threadIdx.x; i < d; i += kThreads) {
-    float pos = 0.f, neg = 0.f;
-    for (int hh = 0; hh < G; ++hh) {
-      const float x = load_elem<E>(a.q, (static_cast<size_t>(b) * a.n_q_heads + g * G + hh) * d + i);
-      pos += fmaxf(x, 0.f);
-      neg += fminf(x, 0.f);
-    }
-    qpm[i] = pos;
-    qpm[d + i] = neg;
+  if constexpr (QFOLD) {  // folded once per group by launch_query_fold
+    const float *src = a.qfold + static_cast<size_t>(group) * 2 * d;
+    for (int i = threadIdx.x; i < 2 * d; i += kThreads) qpm[i] = __ldcg(src + i);
+  } else {
+    fold_query<E, NCH, 8>(a.q, static_cast<size_t>(b) * a.n_q_heads + static_cast<size_t>(g) * G, G, d, qpm);
   }
   __syncthreads();
   float qr[CPL][EPC];
@@ -132,6 +221,17 @@ __device__ __forceinline__ void score_blocks(const BlockScoreArgs &a, int group,
   }
 }
 
+// [Q+; Q-] of group blockIdx.x into a.qfold (one CTA per group).
+template <typename E, int NCH>
+__global__ void __launch_bounds__(kThreads) query_fold_kernel(BlockScoreArgs a) {
+  grid_dependency_wait();
+  const int group = blockIdx.x;
+  const int b = group / a.n_kv_heads, g = group % a.n_kv_heads;
+  const int G = a.n_q_heads / a.n_kv_heads;
+  fold_query<E, NCH, 8>(a.q, static_cast<size_t>(b) * a.n_q_heads + static_cast<size_t>(g) * G, G, a.d,
+                        a.qfold + static_cast<size_t>(group) * 2 * a.d);
+}
+
 // The stage-1 keys of rows [r0, r1) from block scores a previous launch
 // wrote (the two-phase selection): the same keys score_blocks makes.
 __device__ __forceinline__ void keys_from_scores(const BlockScoreArgs &a, int group, int nb, int r0, int r1,
@@ -148,7 +248,7 @@ __device__ __forceinline__ void keys_from_scores(const BlockScoreArgs &a, int gr
 // Phase 1 of the two-phase selection: CTA c scores the c-th equal range of
 // all groups' summary rows (a range may cross into the next group; the
 // query fold is redone per group) into a.scores, with score_blocks' arithmetic.
-template <typename E, int NCH>
+template <typename E, int NCH, bool QFOLD>
 __global__ void __launch_bounds__(kThreads, NCH > 32 ? 2 : 4) block_scores_kernel(BlockScoreArgs a, int rows_per_cta) {
   extern __shared__ float qpm[];  // [2d]
   grid_dependency_wait();
@@ -161,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, NCH > 32 ? 2 : 4) block_scores_kerne
     const long long gend = std::min(r1, gbase + a.n_blocks_max);
     const int sq = min(max(a.seq_lens[group / a.n_kv_heads], 0), a.max_ctx);
     const int nb = (sq + a.block_size - 1) / a.block_size;
-    score_blocks<E, NCH, false>(a, group, nb, static_cast<int>(r0 - gbase), static_cast<int>(gend - gbase), qpm,
+    score_blocks<E, NCH, false, QFOLD>(a, group, nb, static_cast<int>(r0 - gbase), static_cast<int>(gend - gbase), qpm,
                                 nullptr, nullptr);
     __syncthreads();  // qpm is folded again for the next group
     r0 = gend;
@@ -237,17 +337,47 @@ __device__ __forceinline__ void score_blocks_max(const BlockScoreArgs &a, int gr
 
 // Qbar_L[c] = sum_h q_h[L[c]] (fp32, heads in order) into qbar[0..r); with an
 // int8 slab the channel's scale is folded in: qbar[c] = scale_c * Qbar_L[c].
-template <typename E>
+// All threads of the CTA call it.  PAR (the latent rows, many heads): thread
+// t takes label t / P and the heads of part t % P (4 loads in flight) and the
+// part sums are added in part order; otherwise thread c sums label c over the
+// heads in order.  Every kernel of a shape takes the same PAR (d > 128).
+template <typename E, bool PAR>
 __device__ __forceinline__ void fold_label_query(const TokenArgs &a, int group, float *qbar) {
   const int b = group / a.n_kv_heads, g = group % a.n_kv_heads;
   const int G = a.n_q_heads / a.n_kv_heads;
-  for (int c = threadIdx.x; c < a.n_label; c += kThreads) {
-    const int ch = a.label_idx[c];
+  if constexpr (!PAR) {
+    for (int c = threadIdx.x; c < a.n_label; c += kThreads) {
+      const int ch = a.label_idx[c];
+      float sum = 0.f;
+      if (ch >= 0 && ch < a.d)
+        for (int hh = 0; hh < G; ++hh)
+          sum += load_elem<E>(a.q, (static_cast<size_t>(b) * a.n_q_heads + g * G + hh) * a.d + ch);
+      qbar[c] = a.scales ? sum * a.scales[static_cast<size_t>(group) * a.n_label + c] : sum;
+    }
+    return;
+  }
+  const int P = fold_parts(G, a.n_label);
+  const int HP = (G + P - 1) / P;
+  const size_t row0 = static_cast<size_t>(b) * a.n_q_heads + static_cast<size_t>(g) * G;
+  for (int base = 0; base < a.n_label * P; base += kThreads) {
+    const int t = base + static_cast<int>(threadIdx.x);
+    const int c = t / P, part = t % P;
+    const int ch = c < a.n_label ? a.label_idx[c] : -1;
     float sum = 0.f;
-    if (ch >= 0 && ch < a.d)
-      for (int hh = 0; hh < G; ++hh)
-        sum += load_elem<E>(a.q, (static_cast<size_t>(b) * a.n_q_heads + g * G + hh) * a.d + ch);
-    qbar[c] = a.scales ? sum * a.scales[static_cast<size_t>(group) * a.n_label + c] : sum;
+    if (ch >= 0 && ch < a.d) {
+      const int h0 = part * HP, h1 = min(G, h0 + HP);
+      for (int hb = h0; hb < h1; hb += 4) {
+        float x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) x[u] = hb + u < h1 ? load_elem<E>(a.q, (row0 + hb + u) * a.d + ch) : 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (hb + u < h1) sum += x[u];
+      }
+    }
+    const float tot = fold_lanes(sum, P);
+    if (c < a.n_label && part == 0)
+      qbar[c] = a.scales ? tot * a.scales[static_cast<size_t>(group) * a.n_label + c] : tot;
   }
 }
 
@@ -356,7 +486,7 @@ __global__ void __launch_bounds__(kThreads, NCH > 32 ? 2 : 4) block_select_kerne
       [r0](int i) { return r0 + i; }, S, a.err);
 }
 
-template <typename E, typename SE, int RCH, int CS>
+template <typename E, typename SE, int RCH, int CS, bool PAR>
 __global__ void __launch_bounds__(kThreads, token_min_blocks<RCH, SE::kEPC>())
     token_select_kernel(TokenArgs a, int per_cta) {
   extern __shared__ uint32_t keys[];  // [per_cta]
@@ -374,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, token_min_blocks<RCH, SE::kEPC>())
     const int v = a.block_idx[static_cast<size_t>(group) * a.k_b + sl.jb0 + i];
     blk[i] = (v >= 0 && v < a.n_blocks_max) ? v : -1;
   }
-  fold_label_query<E>(a, group, qbar);
+  fold_label_query<E, PAR>(a, group, qbar);
   __syncthreads();
   score_tokens<SE, RCH>(a, group, seq, sl.c0, sl.c1, blk, sl.jb0, qbar, keys, S.hist);
   const int bs = a.block_size, jb0 = sl.jb0, c0 = sl.c0;
@@ -393,10 +523,16 @@ struct StepArgs {
   TokenArgs tok;
 };
 
-template <typename E, typename SE, int NCH, int RCH, int CS>
+// local_n > 0 (block scores in global memory, a.from_scores, at most
+// kLocalBlockKeys blocks): every CTA selects the group's K_b blocks itself from
+// all local_n scores (no cluster exchange); rank 0 writes the block ids.
+constexpr int kLocalBlockKeys = 4096;
+
+template <typename E, typename SE, int NCH, int RCH, int CS, bool LOCAL>
 __global__ void __launch_bounds__(kThreads, NCH > 32 ? 2 : token_min_blocks<RCH, SE::kEPC>())
-    select_step_kernel(StepArgs s, int rows_per_cta, int per_cta) {
-  extern __shared__ float qpm[];  // [2d] Q^+, Q^-; block keys [rows_per_cta]; token keys [per_cta]
+    select_step_kernel(StepArgs s, int rows_per_cta, int per_cta, int local_n) {
+  // dynamic: [max(2d Q^+ Q^- + rows_per_cta block keys, local_n block keys)][per_cta token keys]
+  extern __shared__ float qpm[];
   __shared__ ClusterSelectSmem<CS> SB, ST;
   __shared__ int blk[1024];
   __shared__ float qbar[64];
@@ -408,7 +544,7 @@ __global__ void __launch_bounds__(kThreads, NCH > 32 ? 2 : token_min_blocks<RCH,
   const int group = blockIdx.y;
   const int rank = static_cast<int>(cluster_ctarank());
   uint32_t *bkeys = reinterpret_cast<uint32_t *>(qpm + 2 * a.d);
-  uint32_t *tkeys = bkeys + rows_per_cta;
+  uint32_t *tkeys = reinterpret_cast<uint32_t *>(qpm) + max(2 * a.d + rows_per_cta, local_n);
   if (threadIdx.x < kCBins) {
     SB.hist[threadIdx.x] = 0;
     ST.hist[threadIdx.x] = 0;
@@ -425,24 +561,52 @@ __global__ void __launch_bounds__(kThreads, NCH > 32 ? 2 : token_min_blocks<RCH,
   const int b = group / a.n_kv_heads;
   const int sq = min(max(a.seq_lens[b], 0), a.max_ctx);
   const int nb = (sq + a.block_size - 1) / a.block_size;
-  fold_label_query<E>(t, group, qbar);  // independent of the block stage; complete by the next barrier
-  // ---- stages 1 + 2
-  const int r0 = rank * rows_per_cta;
-  const int r1 = min(r0 + rows_per_cta, a.n_blocks_max);
-  if (a.from_scores) keys_from_scores(a, group, nb, r0, r1, bkeys, SB.hist);
-  else score_blocks<E, NCH>(a, group, nb, r0, r1, qpm, bkeys, SB.hist);
+  fold_label_query<E, (NCH > 64)>(t, group, qbar);  // independent of the block stage; complete by the next barrier
   int32_t *bout = a.block_idx + static_cast<size_t>(group) * a.k_b;
-  cluster_topk<kThreads, CS, kSliceCap>(
-      bkeys, max(r1 - r0, 0), a.k_b, bout, a.k_b, [r0](int i) { return r0 + i; }, SB, a.err);
-  // every CTA's block ids are in global memory and visible to the cluster
-  cluster_arrive_release();
-  cluster_wait();
-  // ---- stages 3 + 4
-  const TokenSlice sl = token_slice(t, rank, per_cta);
-  for (int i = threadIdx.x; i < sl.nblk; i += kThreads) {
-    const int v = __ldcg(bout + sl.jb0 + i);
-    blk[i] = (v >= 0 && v < t.n_blocks_max) ? v : -1;
+  TokenSlice sl;
+  if constexpr (LOCAL) {
+    // ---- stages 1 + 2 from the scores in global memory, in every CTA
+    uint32_t *lkeys = reinterpret_cast<uint32_t *>(qpm);
+    const int nbm = min(local_n, a.n_blocks_max);
+    keys_from_scores(a, group, nb, 0, nbm, lkeys, SB.hist);  // (the cluster histogram stays unused)
+    const int k = cta_topk<kThreads, kLocalBlockKeys>(lkeys, nbm, a.k_b, blk, [](int i) { return i; }, SB.hist,
+                                                      SB.bc, SB.sh);
+    for (int i = max(k, 0) + threadIdx.x; i < a.k_b; i += kThreads) blk[i] = -1;
+    sl = token_slice(t, rank, per_cta);
+    __syncthreads();
+    if (rank == 0)
+      for (int i = threadIdx.x; i < a.k_b; i += kThreads) bout[i] = blk[i];
+    // this CTA's slice of the kept-block list moves to the front of blk
+    int v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = u * kThreads + threadIdx.x;
+      v[u] = i < sl.nblk ? blk[sl.jb0 + i] : -1;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = u * kThreads + threadIdx.x;
+      if (i < sl.nblk) blk[i] = (v[u] >= 0 && v[u] < t.n_blocks_max) ? v[u] : -1;
+    }
+  } else {
+    // ---- stages 1 + 2
+    const int r0 = rank * rows_per_cta;
+    const int r1 = min(r0 + rows_per_cta, a.n_blocks_max);
+    if (a.from_scores) keys_from_scores(a, group, nb, r0, r1, bkeys, SB.hist);
+    else score_blocks<E, NCH>(a, group, nb, r0, r1, qpm, bkeys, SB.hist);
+    cluster_topk<kThreads, CS, kSliceCap>(
+        bkeys, max(r1 - r0, 0), a.k_b, bout, a.k_b, [r0](int i) { return r0 + i; }, SB, a.err);
+    // every CTA's block ids are in global memory and visible to the cluster
+    cluster_arrive_release();
+    cluster_wait();
+    sl = token_slice(t, rank, per_cta);
+    for (int i = threadIdx.x; i < sl.nblk; i += kThreads) {
+      const int v = __ldcg(bout + sl.jb0 + i);
+      blk[i] = (v >= 0 && v < t.n_blocks_max) ? v : -1;
+    }
   }
+  // ---- stages 3 + 4
   __syncthreads();
   score_tokens<SE, RCH>(t, group, sq, sl.c0, sl.c1, blk, sl.jb0, qbar, tkeys, ST.hist);
   const int bs = t.block_size, jb0 = sl.jb0, c0 = sl.c0;
@@ -453,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, NCH > 32 ? 2 : token_min_blocks<RCH,
         const int jb = j / bs;
         return blk[jb - jb0] * bs + (j - jb * bs);
       },
-      ST, t.err, /*entry_wait=*/false);
+      ST, t.err, /*entry_wait=*/LOCAL);
   if (t.ready) {  // every CTA's token ids are written: the group is ready for its attention
     __threadfence();
     cluster_arrive_release();
@@ -506,11 +670,11 @@ cudaError_t run_token_select(const TokenArgs &a, cudaStream_t st) {
   constexpr int CS = kClusterSize;
   const int per = (a.k_b * a.block_size + CS - 1) / CS;  // <= kSliceCap
   const size_t smem = static_cast<size_t>(per) * sizeof(uint32_t);
-  static int allowed[64] = {};
-  cudaError_t e = allow_smem(token_select_kernel<E, SE, RCH, CS>, smem, allowed);
+  auto kern = a.d > 128 ? token_select_kernel<E, SE, RCH, CS, true> : token_select_kernel<E, SE, RCH, CS, false>;
+  static int allowed[2][64] = {};
+  cudaError_t e = allow_smem(kern, smem, allowed[a.d > 128]);
   if (e != cudaSuccess) return e;
-  return launch_pdl_cluster(token_select_kernel<E, SE, RCH, CS>, dim3(CS, a.batch * a.n_kv_heads), dim3(kThreads), smem,
-                            st, CS, a, per);
+  return launch_pdl_cluster(kern, dim3(CS, a.batch * a.n_kv_heads), dim3(kThreads), smem, st, CS, a, per);
 }
 
 template <typename E, typename SE, int NCH, int RCH>
@@ -518,14 +682,15 @@ cudaError_t run_select_step(const BlockScoreArgs &a, const TokenArgs &t, cudaStr
   constexpr int CS = kClusterSize;
   const int rows = (a.n_blocks_max + CS - 1) / CS;
   const int per = (t.k_b * t.block_size + CS - 1) / CS;
-  const size_t smem = 2 * static_cast<size_t>(a.d) * sizeof(float) +
-                      (static_cast<size_t>(rows) + static_cast<size_t>(per)) * sizeof(uint32_t);
-  auto kern = select_step_kernel<E, SE, NCH, RCH, CS>;
-  static int allowed[64] = {};
-  cudaError_t e = allow_smem(kern, smem, allowed);
+  const int local_n = a.from_scores && a.n_blocks_max <= kLocalBlockKeys ? a.n_blocks_max : 0;
+  const size_t head = std::max<size_t>(2 * static_cast<size_t>(a.d) + rows, static_cast<size_t>(local_n));
+  const size_t smem = (head + static_cast<size_t>(per)) * sizeof(uint32_t);
+  auto kern = local_n > 0 ? select_step_kernel<E, SE, NCH, RCH, CS, true> : select_step_kernel<E, SE, NCH, RCH, CS, false>;
+  static int allowed[2][64] = {};
+  cudaError_t e = allow_smem(kern, smem, allowed[local_n > 0]);
   if (e != cudaSuccess) return e;
   return launch_pdl_cluster(kern, dim3(CS, a.batch * a.n_kv_heads), dim3(kThreads), smem, st, CS, StepArgs{a, t},
-                            rows, per);
+                            rows, per, local_n);
 }
 
 template <typename E, int NCH>
@@ -589,14 +754,25 @@ cudaError_t launch_token_select(const TokenArgs &a, cudaStream_t st) {
   return cudaErrorInvalidValue;
 }
 
-bool select_two_phase(int groups, int heads_per_group, int num_sms, size_t summary_bytes) {
+bool select_two_phase(int groups, int heads_per_group, int num_sms, size_t summary_bytes, bool folded_queries) {
   // One cluster of kClusterSize CTAs per group: with fewer clusters than fill
   // the SMs twice over, the summary stream is short of loads in flight.  Below
-  // a few MB of summary the extra launch costs more than it saves, and with
-  // many heads per group every phase-1 CTA pays the query fold over all of
-  // them (measured: gqa48k 21.9 -> 18.4 us; the 64-head latent 33.8 -> 37.7 us).
+  // a few MB of summary the extra launch costs more than it saves.  With many
+  // heads per group the queries must be folded once per group beforehand
+  // (launch_query_fold): folded by every phase-1 CTA, the fold costs more than
+  // the stream (measured: gqa48k 21.9 -> 18.4 us; the 64-head latent
+  // 33.8 -> 37.7 us without the separate fold).
   return static_cast<long long>(groups) * kClusterSize < 2LL * num_sms && summary_bytes >= (size_t(4) << 20) &&
-         heads_per_group <= 16;
+         (heads_per_group <= 16 || folded_queries);
+}
+
+cudaError_t launch_query_fold(const BlockScoreArgs &a, cudaStream_t st) {
+  if (!a.qfold) return cudaErrorInvalidValue;
+  const dim3 grid(a.batch * a.n_kv_heads);
+  if (a.dtype == 1)  // the fold of score_blocks<BF16, NCH>: sequential below NCH 64, parallel above
+    return a.d > 128 ? launch_pdl(query_fold_kernel<BF16, 144>, grid, dim3(kThreads), 0, st, a)
+                     : launch_pdl(query_fold_kernel<BF16, 32>, grid, dim3(kThreads), 0, st, a);
+  return launch_pdl(query_fold_kernel<F32, 32>, grid, dim3(kThreads), 0, st, a);
 }
 
 namespace {
@@ -607,7 +783,8 @@ cudaError_t run_block_scores(const BlockScoreArgs &a, int num_sms, cudaStream_t 
   const int rows = static_cast<int>((total + ctas - 1) / ctas);
   const int grid = static_cast<int>((total + rows - 1) / rows);
   const size_t smem = 2 * static_cast<size_t>(a.d) * sizeof(float);
-  return launch_pdl(block_scores_kernel<E, NCH>, dim3(grid), dim3(kThreads), smem, st, a, rows);
+  if (a.qfold) return launch_pdl(block_scores_kernel<E, NCH, true>, dim3(grid), dim3(kThreads), smem, st, a, rows);
+  return launch_pdl(block_scores_kernel<E, NCH, false>, dim3(grid), dim3(kThreads), smem, st, a, rows);
 }
 }  // namespace
 
