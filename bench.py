@@ -82,7 +82,8 @@ def read_peaks() -> dict:
 # valid while these are unchanged)
 STAGE_SOURCES = {
     "stage_select": ["tls_select.cu", "tls_device.cuh", "tls_internal.h"],
-    "stage_attn": ["tls_attn.cu", "tls_attn_mma.cu", "tls_mma.cuh", "tls_device.cuh", "tls_internal.h"],
+    "stage_attn": ["tls_attn.cu", "tls_attn_mma.cu", "tls_attn_mla_tc.cu", "tls_mma.cuh", "tls_device.cuh",
+                   "tls_internal.h"],
 }
 
 
@@ -269,10 +270,13 @@ def gpu_arm(args, rank, world, local_rank):
     # stages 1-4 (one cluster launch; with few groups a block-score launch
     # first), attention split, log-sum-exp merge
     groups = w.batch * w.n_kv_heads
-    two_phase = (groups * 8 < 2 * torch.cuda.get_device_properties(dev).multi_processor_count
-                 and algorithmic_bytes(w)["block_summary"] >= 4 << 20 and w.group <= 16)
-    # max-over-heads: a score launch (or the two separate selection launches) before the rest
-    launches_per_step = 3 + (1 if (two_phase or w.block_agg == 1) else 0)
+    # tls_decode_step's launches: with few groups and >= 4 MB of summary the
+    # two-phase selection adds a phase-1 launch (and, for groups of more than
+    # 16 heads, a query-fold launch before it); max-over-heads adds a score
+    # launch (or the two separate selection launches) before the rest
+    two_phase = (w.block_agg == 0 and groups * 8 < 2 * torch.cuda.get_device_properties(dev).multi_processor_count
+                 and algorithmic_bytes(w)["block_summary"] >= 4 << 20)
+    launches_per_step = 3 + (1 if (two_phase or w.block_agg == 1) else 0) + (1 if two_phase and w.group > 16 else 0)
     # The clock sampler starts (and settles) before the warm-up, so that the
     # GPU does not sit idle between the warm-up and the timed region and the
     # timed steps start at the clocks the warm-up brought it to.

@@ -423,10 +423,11 @@ static tls_status select_step_impl(const tls_shape *s, const void *q, const void
   float *scores = block_score_out ? block_score_out : scratch;
   const size_t summary_bytes = static_cast<size_t>(s->batch) * s->n_kv_heads * n_blocks_max(s) * 2 * s->d_qk *
                                (s->kv_dtype == TLS_BF16 ? 2 : 4);
-  if (scores && tls::select_two_phase(s->batch * s->n_kv_heads, s->n_q_heads / s->n_kv_heads, device_sms(),
-                                      summary_bytes, qfold != nullptr)) {
+  const int G = s->n_q_heads / s->n_kv_heads;
+  if (G <= 16) qfold = nullptr;  // a few heads: each phase-1 CTA folds them faster than an extra launch
+  if (scores && tls::select_two_phase(s->batch * s->n_kv_heads, G, device_sms(), summary_bytes, qfold != nullptr)) {
     a.scores = scores;
-    if (qfold) {  // the queries folded once per group, not by every phase-1 CTA
+    if (qfold) {  // many heads: the queries folded once per group, not by every phase-1 CTA
       a.qfold = qfold;
       st = cuda_status(tls::launch_query_fold(a, cs), "query_fold launch");
       if (st != TLS_OK) return st;
