@@ -255,14 +255,14 @@ def gpu_arm(args, rank, world, local_rank):
         T.tls_decode_step(shape, L.q, L.meta, L.slab, label, seq_lens, L.K, L.V, bidx, tidx, out, lse, None, None,
                           ws, sh)
 
-    bscore = torch.empty((G, w.n_blocks), dtype=torch.float32, device=dev)
 
     def step_stages(L, ev):
-        """The same step as its two calls, with CUDA events around each (the
-        selection given a block-score buffer, as tls_decode_step gives it
-        workspace, so that it runs the same launches)."""
+        """The same step as its two calls, with CUDA events around each: the
+        selection with tls_decode_step's workspace (tls_select_step_ws, the
+        same launches as the selection part of tls_decode_step), then the
+        attention."""
         ev[0].record(stream)
-        T.tls_select_step(shape, L.q, L.meta, L.slab, label, seq_lens, bidx, tidx, bscore, None, sh)
+        T.tls_select_step_ws(shape, L.q, L.meta, L.slab, label, seq_lens, bidx, tidx, ws, None, None, sh)
         ev[1].record(stream)
         T.tls_sparse_attn_decode(shape, L.q, L.K, L.V, tidx, out, lse, ws, sh)
         ev[2].record(stream)
@@ -422,7 +422,7 @@ def gpu_arm(args, rank, world, local_rank):
         "stages_us": {n: float(v * 1e3) for n, v in zip(names, stage_ms)},
         "stages_median_us": {n: float(v * 1e3) for n, v in zip(names, stage_med)},
         "stage_timing": f"separate untimed pass of {n_stage} steps after the timed region: the step as its two "
-                        f"calls (tls_select_step, tls_sparse_attn_decode), CUDA events around each on every step "
+                        f"calls (tls_select_step_ws, tls_sparse_attn_decode), CUDA events around each on every step "
                         f"(first step dropped); mean reported",
         "step_call": "tls_decode_step",
         "roofline": {

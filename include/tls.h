@@ -232,6 +232,18 @@ TLS_API tls_status tls_select_step(const tls_shape *s, const void *q, const void
                                    int32_t *token_idx_out, float *block_score_out, float *token_score_out,
                                    void *stream);
 
+/* tls_select_step with tls_decode_step's workspace (ws: at least
+ * tls_workspace_size(s) bytes, 256-byte aligned; checked before anything is
+ * enqueued): the same launches as the selection part of tls_decode_step, so
+ * that the selection can be run and timed on its own.  The two-phase
+ * selection keeps the block scores in ws unless block_score_out is given, and
+ * for more than 16 heads per group folds the queries into ws once per group.
+ * Ids and scores are the same bits as tls_select_step's. */
+TLS_API tls_status tls_select_step_ws(const tls_shape *s, const void *q, const void *meta, const void *slab,
+                                      const int32_t *label_idx, const int32_t *seq_lens, int32_t *block_idx_out,
+                                      int32_t *token_idx_out, float *block_score_out, float *token_score_out, void *ws,
+                                      size_t ws_bytes, void *stream);
+
 /* Stages 1-5 in one call: tls_select_step, then tls_sparse_attn_decode on its
  * token ids, for callers that want the whole decode step.  Its two-phase
  * selection (few groups, as in tls_select_step, the block scores in the

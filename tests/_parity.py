@@ -328,6 +328,21 @@ def full_stage_parity(w: W.Workload, seq_lens=None, out_dtype=0, name=None, inp=
                 step_swaps_t += check_selection(ft[b, g], orc.cand_tok[b, g][oko], orc.cand_scores[b, g][oko], w.k_t,
                                                 what + " tokens")
             check_selection_self_consistent(ft[b, g], cand[ok].astype(np.int32), fts[b, g][ok], what + " tokens")
+    # the same selection with tls_decode_step's workspace (its launches: the
+    # two-phase path may fold the queries once and select the blocks per CTA):
+    # the same bits
+    wb = torch.full_like(torch.from_numpy(fb), -7).cuda()
+    wt = torch.full_like(torch.from_numpy(ft), -7).cuda()
+    wbs = torch.zeros(fbs.shape, dtype=torch.float32, device="cuda")
+    wts = torch.zeros(fts.shape, dtype=torch.float32, device="cuda")
+    tls().tls_select_step_ws(gpu.shape, gpu.q, gpu.meta, gpu.slab, gpu.label, gpu.seq_lens, wb, wt, gpu.ws, wbs, wts)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(wb.cpu().numpy(), fb, err_msg=f"{name} select_step_ws block ids")
+    np.testing.assert_array_equal(wt.cpu().numpy(), ft, err_msg=f"{name} select_step_ws token ids")
+    np.testing.assert_array_equal(wbs.cpu().numpy().view(np.uint32), fbs.view(np.uint32),
+                                  err_msg=f"{name} select_step_ws block scores")
+    np.testing.assert_array_equal(wts.cpu().numpy().view(np.uint32), fts.view(np.uint32),
+                                  err_msg=f"{name} select_step_ws token scores")
     # stages 1-5 in one call (tls_decode_step, the call the benchmark times):
     # block / token ids and both score arrays identical to the select_step
     # launch above, attention against the oracle wherever the token ids equal

@@ -181,6 +181,19 @@ def test_select_step_checks_before_launch(T):
     assert st == T.TLS_ERR_UNSUPPORTED
 
 
+def test_select_step_ws_checks_before_launch(T):
+    s = good_shape(T)
+    need = T.tls_workspace_size(s)
+    # workspace missing, too small or misaligned: refused before anything else
+    for ws, nbytes in ((None, need), (256, need - 1), (0x1010, need)):
+        st = T._lib.tls_select_step_ws(ctypes.byref(s), 256, 256, 256, 256, 256, 256, 256, None, None, ws, nbytes,
+                                       None)
+        assert st == T.TLS_ERR_WORKSPACE and str(need) in T.tls_last_error()
+    # then the pointers, as tls_select_step checks them
+    st = T._lib.tls_select_step_ws(ctypes.byref(s), 256, 256, None, 256, 256, 256, 256, None, None, 256, need, None)
+    assert st == T.TLS_ERR_INVALID_ARG and "slab is NULL" in T.tls_last_error()
+
+
 def test_append_tokens_checks_before_launch(T):
     s = good_shape(T)
     assert T._lib.tls_append_tokens(ctypes.byref(s), 256, 256, 256, -1, 256, 256, None, None) == T.TLS_ERR_INVALID_ARG

@@ -439,6 +439,22 @@ static tls_status select_step_impl(const tls_shape *s, const void *q, const void
   return cuda_status(tls::launch_select_step(a, t, cs), "select_step launch");
 }
 
+tls_status tls_select_step_ws(const tls_shape *s, const void *q, const void *meta, const void *slab,
+                              const int32_t *label_idx, const int32_t *seq_lens, int32_t *block_idx_out,
+                              int32_t *token_idx_out, float *block_score_out, float *token_score_out, void *ws,
+                              size_t ws_bytes, void *stream) {
+  tls_status st = check_shape(s);
+  if (st != TLS_OK) return st;
+  if (s->batch == 0) return TLS_OK;
+  const size_t need = tls_workspace_size(s);
+  if (!need) return fail(TLS_ERR_UNSUPPORTED, "no workspace layout for this shape");
+  if (!ws || ws_bytes < need || !aligned(ws, 256))
+    return fail(TLS_ERR_WORKSPACE, "workspace too small or not 256-byte aligned (need %zu bytes)", need);
+  return select_step_impl(s, q, meta, slab, label_idx, seq_lens, block_idx_out, token_idx_out, block_score_out,
+                          token_score_out, static_cast<float *>(ws),
+                          reinterpret_cast<float *>(static_cast<char *>(ws) + fold_offset(s)), nullptr, 0, stream);
+}
+
 static tls_status attn_common(const tls_shape *s, const void *q, const void *K, const void *V,
                               const int32_t *token_idx, const int32_t *slot_of_block, int32_t n_slots, void *out,
                               float *lse_out, void *ws, size_t ws_bytes, void *stream, bool paged,

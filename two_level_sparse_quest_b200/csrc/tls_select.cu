@@ -66,19 +66,23 @@ __device__ __forceinline__ float fold_lanes(float v, int P) {
 // the heads of part t % P (consecutive heads, 8 loads in flight); the P part
 // sums are then added in part order.  With P = G (small groups) the sums are
 // the sequential sums over the heads.  FB: loads in flight per thread.
+// Chunk columns [c_begin, c_end) only (a fold split over several CTAs), by
+// the CTA's nthr threads; P depends on G and d alone, so every split gives the
+// same bits.
 template <typename E, int FB>
-__device__ __forceinline__ void fold_group_query(const void *q, size_t row0, int G, int d, float *qpm) {
+__device__ __forceinline__ void fold_group_query(const void *q, size_t row0, int G, int d, float *qpm,
+                                                 int c_begin, int c_end, int nthr) {
   constexpr int EPC = E::kEPC;
   const int NC = d / EPC;
   const int P = fold_parts(G, NC);
   const int HP = (G + P - 1) / P;
-  for (int base = 0; base < NC * P; base += kThreads) {  // one pass unless NC > kThreads
+  for (int base = c_begin * P; base < c_end * P; base += nthr) {
     const int t = base + static_cast<int>(threadIdx.x);
     const int c = t / P, part = t % P;
     float pos[EPC], neg[EPC];
 #pragma unroll
     for (int e = 0; e < EPC; ++e) pos[e] = neg[e] = 0.f;
-    if (c < NC) {
+    if (c < c_end) {
       const uint4 *src = static_cast<const uint4 *>(q) + row0 * NC + c;
       const int h0 = part * HP, h1 = min(G, h0 + HP);
       for (int hb = h0; hb < h1; hb += FB) {
@@ -102,7 +106,7 @@ __device__ __forceinline__ void fold_group_query(const void *q, size_t row0, int
 #pragma unroll
     for (int e = 0; e < EPC; ++e) {
       const float sp = fold_lanes(pos[e], P), sn = fold_lanes(neg[e], P);
-      if (c < NC && part == 0) {
+      if (c < c_end && part == 0) {
         qpm[c * EPC + e] = sp;
         qpm[d + c * EPC + e] = sn;
       }
@@ -117,7 +121,7 @@ __device__ __forceinline__ void fold_group_query(const void *q, size_t row0, int
 template <typename E, int NCH, int FB>
 __device__ __forceinline__ void fold_query(const void *q, size_t row0, int G, int d, float *qpm) {
   if constexpr (NCH > 64) {
-    fold_group_query<E, FB>(q, row0, G, d, qpm);
+    fold_group_query<E, FB>(q, row0, G, d, qpm, 0, d / E::kEPC, kThreads);
   } else {
     for (int i = threadIdx.x; i < d; i += kThreads) {
       float pos = 0.f, neg = 0.f;
@@ -221,15 +225,25 @@ __device__ __forceinline__ void score_blocks(const BlockScoreArgs &a, int group,
   }
 }
 
-// [Q+; Q-] of group blockIdx.x into a.qfold (one CTA per group).
+// [Q+; Q-] of group blockIdx.x into a.qfold.  d <= 128: one CTA per group,
+// the per-channel fold.  Latent rows: blockIdx.y takes 8 of the 72 chunk
+// columns (one warp, every head of a part in flight at once), so the fold of
+// a group is one round trip of 72 KB spread over 9 CTAs.
 template <typename E, int NCH>
-__global__ void __launch_bounds__(kThreads) query_fold_kernel(BlockScoreArgs a) {
+__global__ void __launch_bounds__(NCH > 64 ? 32 : kThreads) query_fold_kernel(BlockScoreArgs a) {
   grid_dependency_wait();
   const int group = blockIdx.x;
   const int b = group / a.n_kv_heads, g = group % a.n_kv_heads;
   const int G = a.n_q_heads / a.n_kv_heads;
-  fold_query<E, NCH, 8>(a.q, static_cast<size_t>(b) * a.n_q_heads + static_cast<size_t>(g) * G, G, a.d,
-                        a.qfold + static_cast<size_t>(group) * 2 * a.d);
+  const size_t row0 = static_cast<size_t>(b) * a.n_q_heads + static_cast<size_t>(g) * G;
+  float *dst = a.qfold + static_cast<size_t>(group) * 2 * a.d;
+  if constexpr (NCH > 64) {
+    const int NC = a.d / E::kEPC;
+    const int c0 = blockIdx.y * 8, c1 = min(NC, c0 + 8);
+    fold_group_query<E, 32>(a.q, row0, G, a.d, dst, c0, c1, 32);
+  } else {
+    fold_query<E, NCH, 8>(a.q, row0, G, a.d, dst);
+  }
 }
 
 // The stage-1 keys of rows [r0, r1) from block scores a previous launch
@@ -682,7 +696,15 @@ cudaError_t run_select_step(const BlockScoreArgs &a, const TokenArgs &t, cudaStr
   constexpr int CS = kClusterSize;
   const int rows = (a.n_blocks_max + CS - 1) / CS;
   const int per = (t.k_b * t.block_size + CS - 1) / CS;
-  const int local_n = a.from_scores && a.n_blocks_max <= kLocalBlockKeys ? a.n_blocks_max : 0;
+  // each CTA selecting the blocks itself pays off while the clusters do not
+  // fill the GPU (few groups); with many groups the cluster exchange is cheaper
+  int sms = 148;
+  {
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  }
+  const bool few_groups = static_cast<long long>(a.batch) * a.n_kv_heads * CS < 2LL * sms;
+  const int local_n = a.from_scores && few_groups && a.n_blocks_max <= kLocalBlockKeys ? a.n_blocks_max : 0;
   const size_t head = std::max<size_t>(2 * static_cast<size_t>(a.d) + rows, static_cast<size_t>(local_n));
   const size_t smem = (head + static_cast<size_t>(per)) * sizeof(uint32_t);
   auto kern = local_n > 0 ? select_step_kernel<E, SE, NCH, RCH, CS, true> : select_step_kernel<E, SE, NCH, RCH, CS, false>;
@@ -768,18 +790,19 @@ bool select_two_phase(int groups, int heads_per_group, int num_sms, size_t summa
 
 cudaError_t launch_query_fold(const BlockScoreArgs &a, cudaStream_t st) {
   if (!a.qfold) return cudaErrorInvalidValue;
-  const dim3 grid(a.batch * a.n_kv_heads);
-  if (a.dtype == 1)  // the fold of score_blocks<BF16, NCH>: sequential below NCH 64, parallel above
-    return a.d > 128 ? launch_pdl(query_fold_kernel<BF16, 144>, grid, dim3(kThreads), 0, st, a)
-                     : launch_pdl(query_fold_kernel<BF16, 32>, grid, dim3(kThreads), 0, st, a);
-  return launch_pdl(query_fold_kernel<F32, 32>, grid, dim3(kThreads), 0, st, a);
+  const unsigned groups = static_cast<unsigned>(a.batch * a.n_kv_heads);
+  if (a.dtype == 1 && a.d > 128)  // the fold of score_blocks<BF16, 144>: parallel, 8 chunk columns per CTA
+    return launch_pdl(query_fold_kernel<BF16, 144>, dim3(groups, (a.d / 8 + 7) / 8), dim3(32), 0, st, a);
+  if (a.dtype == 1) return launch_pdl(query_fold_kernel<BF16, 32>, dim3(groups), dim3(kThreads), 0, st, a);
+  return launch_pdl(query_fold_kernel<F32, 32>, dim3(groups), dim3(kThreads), 0, st, a);
 }
 
 namespace {
 template <typename E, int NCH>
 cudaError_t run_block_scores(const BlockScoreArgs &a, int num_sms, cudaStream_t st) {
   const long long total = static_cast<long long>(a.batch) * a.n_kv_heads * a.n_blocks_max;
-  const int ctas = static_cast<int>(std::max<long long>(1, std::min<long long>(4LL * num_sms, total)));
+  // one wave: the kernel's resident CTAs per SM (2 for the latent rows' 128 registers, else 4)
+  const int ctas = static_cast<int>(std::max<long long>(1, std::min<long long>((NCH > 32 ? 2LL : 4LL) * num_sms, total)));
   const int rows = static_cast<int>((total + ctas - 1) / ctas);
   const int grid = static_cast<int>((total + rows - 1) / rows);
   const size_t smem = 2 * static_cast<size_t>(a.d) * sizeof(float);

@@ -31,7 +31,7 @@ STATUS_NAMES = {0: "TLS_OK", 1: "TLS_ERR_INVALID_ARG", 2: "TLS_ERR_UNSUPPORTED",
 EXPORTED = ("tls_version", "tls_last_error", "tls_workspace_size", "tls_build_block_meta", "tls_block_score_topk",
             "tls_token_score_topk", "tls_sparse_attn_decode", "tls_sparse_attn_decode_paged", "tls_offload_reset",
             "tls_prefetch_diff", "tls_wait_event", "tls_block_score_topk_noalloc", "tls_device_error", "tls_select_step",
-            "tls_append_tokens", "tls_slab_bytes", "tls_noalloc_read_scores", "tls_decode_step")
+            "tls_append_tokens", "tls_slab_bytes", "tls_noalloc_read_scores", "tls_decode_step", "tls_select_step_ws")
 
 
 class TlsShape(ctypes.Structure):
@@ -74,6 +74,7 @@ _sigs = {
     "tls_slab_bytes": ([_S], _sz),
     "tls_noalloc_read_scores": ([_P, _sz, _P], ctypes.c_int),
     "tls_decode_step": ([_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _sz, _P], ctypes.c_int),
+    "tls_select_step_ws": ([_S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _sz, _P], ctypes.c_int),
 }
 for _name, (_args, _ret) in _sigs.items():
     _f = getattr(_lib, _name)
@@ -205,6 +206,17 @@ def tls_select_step(shape, q, meta, slab, label_idx, seq_lens, block_idx_out, to
     _check(_lib.tls_select_step(ctypes.byref(shape), _dptr(q), _dptr(meta), _dptr(slab), _dptr(label_idx),
                                 _dptr(seq_lens), _dptr(block_idx_out), _dptr(token_idx_out), _dptr(block_score_out),
                                 _dptr(token_score_out), _stream(stream)), "tls_select_step")
+
+
+def tls_select_step_ws(shape, q, meta, slab, label_idx, seq_lens, block_idx_out, token_idx_out, ws,
+                       block_score_out=None, token_score_out=None, stream=None):
+    """tls_select_step with tls_decode_step's workspace (the same launches as
+    the selection part of tls_decode_step)."""
+    wp, wn = _ws(ws)
+    _check(_lib.tls_select_step_ws(ctypes.byref(shape), _dptr(q), _dptr(meta), _dptr(slab), _dptr(label_idx),
+                                   _dptr(seq_lens), _dptr(block_idx_out), _dptr(token_idx_out),
+                                   _dptr(block_score_out), _dptr(token_score_out), wp, wn, _stream(stream)),
+           "tls_select_step_ws")
 
 
 def tls_decode_step(shape, q, meta, slab, label_idx, seq_lens, K, V, block_idx_out, token_idx_out, out, lse_out=None,
