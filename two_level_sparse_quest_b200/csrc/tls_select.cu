@@ -193,6 +193,7 @@ __device__ __forceinline__ void score_blocks(const BlockScoreArgs &a, int group,
     uint4 nv[U][CPL];
     const bool more = rb + STEP * U < r1;
     if (more) load_rows(rb + STEP * U, nv);  // next rows in flight during this batch's math
+    float x[U];  // this lane's part of each of the batch's U rows
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       float acc = 0.f;
@@ -203,10 +204,38 @@ __device__ __forceinline__ void score_blocks(const BlockScoreArgs &a, int group,
 #pragma unroll
         for (int e = 0; e < EPC; ++e) acc = fmaf(qr[j][e], f[e], acc);
       }
+      x[u] = acc;
+    }
+    // The U row sums over the row group's LPR lanes in one butterfly: at each
+    // of the first log2(U) steps a lane keeps half of its rows (the upper half
+    // when its lane bit is set) and adds its partner's part of them, the other
+    // steps add the partner's whole sum.  Afterwards lane cl holds the sum of
+    // row u(cl) (its lane bits from the top); the first lane of each row
+    // writes the key, so a batch's key writes and histogram adds run in one
+    // pass over U lanes instead of one lane per row.
+    int u_mine = 0;
 #pragma unroll
-      for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      const int row = rb + u * STEP + sub;
-      if (cl == 0 && row < r1) {
+    for (int o = LPR / 2, R = U; o > 0; o >>= 1) {
+      if (R > 1) {
+        const bool up = (cl & o) != 0;
+#pragma unroll
+        for (int k = 0; k < U / 2; ++k) {
+          if (k < R / 2) {
+            const float send = up ? x[k] : x[k + R / 2];
+            const float recv = __shfl_xor_sync(0xffffffffu, send, o);
+            x[k] = (up ? x[k + R / 2] : x[k]) + recv;
+          }
+        }
+        R /= 2;
+        u_mine = 2 * u_mine + (up ? 1 : 0);
+      } else {
+        x[0] += __shfl_xor_sync(0xffffffffu, x[0], o);
+      }
+    }
+    {
+      const int row = rb + u_mine * STEP + sub;
+      if ((cl % (LPR / U)) == 0 && row < r1) {
+        const float acc = x[0];
         const bool valid = row < nb;
         if constexpr (KEYS) {
           const uint32_t key = valid ? max(score_key(acc), 1u) : 0u;
