@@ -54,6 +54,10 @@ SMALL = {
                 [3001, 4096]),
     "mla_ranges_cross_groups": (W.WORKLOADS["mla64k_b4_bf16"].with_(batch=6, ctx=8192, k_b=24, k_t=1100, n_needles=8),
                                 [8192, 5000, 33, 8192, 1, 7000]),
+    # 16 tiles of 32 tokens per group, one per CTA, and a second sequence
+    # whose short length leaves most of its CTAs without a valid token
+    "mla_one_tile_per_cta": (W.WORKLOADS["mla64k_b4_bf16"].with_(batch=2, ctx=4096, k_b=16, k_t=512, n_needles=4),
+                             [4096, 200]),
     # shape sweep: MHA (one query head per KV head) and MQA (one KV head for
     # 16, 32 or 64 query heads: units of 16 heads on the warp-MMA kernel)
     "mha_h16": (W.WORKLOADS["gqa48k_bf16"].with_(n_q_heads=16, n_kv_heads=16, ctx=2048, k_b=16, k_t=200), None),
@@ -84,7 +88,8 @@ def sharpened(inp, factor):
     return inp
 
 
-@pytest.mark.parametrize("name,factor", [("mla_ranges_cross_groups", 16.0), ("mla_small", 64.0)])
+@pytest.mark.parametrize("name,factor", [("mla_ranges_cross_groups", 16.0), ("mla_small", 64.0),
+                                         ("mla_one_tile_per_cta", 64.0)])
 def test_latent_attention_sharp_softmax(name, factor):
     """Large score spreads: the latent kernel's reference max moves and the
     running output is rescaled inside a CTA's range."""
