@@ -7,7 +7,8 @@
 // score is the largest of the G bounds.  Unlike the sum over heads (which
 // folds into one query vector), the G bounds are a real contraction:
 //   U[blocks x G] = [max_j ; min_j]  .  [q_h^+ ; q_h^-]^T      (K = 2 d)
-// One CTA (one warpgroup) per SM walks (group, 128-block tile) work items:
+// One CTA (one warpgroup; two per SM for d <= 128) walks a contiguous range of
+// (group, 128-block tile) work items:
 //   A = the tile's 128 summary rows, K-major, staged 64 channels (128 B) at a
 //       time into a ring of 128B-swizzled 16 KB regions by 16-byte cp.async;
 //   B = [q^+ ; q^-] of the group's heads as bf16 rows (exact: each element is
@@ -288,7 +289,10 @@ cudaError_t run_score_tc(const BlockScoreArgs &a, int num_sms, cudaStream_t st) 
   }
   const long long items = static_cast<long long>(a.batch) * a.n_kv_heads * ((a.n_blocks_max + kSTile - 1) / kSTile);
   if (items <= 0 || items > (1LL << 30)) return cudaErrorInvalidValue;
-  const int per = static_cast<int>((items + num_sms - 1) / num_sms);  // contiguous items per CTA
+  // two warpgroups per SM where their shared memory fits (d <= 128), so that
+  // twice the summary bytes are in flight; the latent rows' B leaves room for one
+  const int ctas = smem <= 113 * 1024 ? 2 * num_sms : num_sms;
+  const int per = static_cast<int>((items + ctas - 1) / ctas);  // contiguous items per CTA
   const int grid = static_cast<int>((items + per - 1) / per);
   return launch_pdl(kern, dim3(grid), dim3(kSThreads), static_cast<size_t>(smem), st, a, static_cast<int>(items), per);
 }
